@@ -1,0 +1,257 @@
+"""Python binding of libqlora_nf4.so, the B200 (sm_100a) QLoRA NF4 library.
+
+Argument marshalling only: every step of the codec and of the linear layer runs in the library's CUDA
+kernels. PyTorch provides device memory and the current stream. The names follow the C ABI in
+include/qlora_nf4.h:
+
+    quantize(w)                      -> NF4Weight     (qlora_nf4_quantize)
+    dequantize(q, dtype)             -> tensor        (qlora_nf4_dequantize)
+    linear_fwd(X, q, A, B, alpha)    -> (Y, U)        (qlora_linear_fwd)
+    linear_bwd(dY, X, q, A, B, alpha, U) -> (dX, dA, dB)   (qlora_linear_bwd)
+
+The shared library is loaded on first use (so that the build step, a submodule of this package, can run
+before it exists); a call made while it is not built raises ImportError. There is no fallback
+implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqlora_nf4.so")
+
+QLORA_F32, QLORA_BF16 = 0, 1
+STATUS_NONFINITE, STATUS_TIMEOUT = 1, 2
+PROF_NAMES = ("quantize", "dequantize", "fwd_gemm", "bwd_gemm", "lora")
+
+
+class _NF4Struct(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("absmax_e4m3", ctypes.c_void_p),
+                ("scale2", ctypes.c_void_p), ("offset", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
+
+
+_LIB = None
+
+
+def load() -> ctypes.CDLL:
+    """The loaded library (loads it on the first call)."""
+    global _LIB
+    if _LIB is None:
+        _LIB = _open()
+    return _LIB
+
+
+def __getattr__(name):          # `bit_nf4_quantized_14_b200.lib` is the loaded CDLL
+    if name == "lib":
+        return load()
+    raise AttributeError(name)
+
+
+def _open() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m bit_nf4_quantized_14_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i64, sz, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+    P = ctypes.POINTER
+    sig = {
+        "qlora_nf4_codebook": [P(ctypes.c_float), P(ctypes.c_float)],
+        "qlora_nf4_storage_bytes": [i64, P(sz), P(sz), P(sz), P(sz)],
+        "qlora_nf4_quantize_workspace": [i64, P(sz)],
+        "qlora_nf4_quantize": [vp, i32, i64, i64, P(_NF4Struct), vp, sz, vp],
+        "qlora_nf4_dequantize": [P(_NF4Struct), vp, i32, vp],
+        "qlora_linear_workspace": [i64, i64, i64, i32, P(sz)],
+        "qlora_linear_fwd": [vp, i64, P(_NF4Struct), vp, vp, i32, ctypes.c_float, vp, vp, vp, sz, vp],
+        "qlora_linear_bwd": [vp, vp, i64, P(_NF4Struct), vp, vp, i32, ctypes.c_float, vp, vp, vp, vp,
+                             vp, sz, vp],
+        "qlora_get_status": [P(i32), vp],
+        "qlora_error_string": [i32],
+        "qlora_profile_enable": [i32],
+        "qlora_profile_read": [P(i64), P(ctypes.c_double)],
+        "qlora_kernel_launches": [],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = {"qlora_error_string": ctypes.c_char_p, "qlora_kernel_launches": i64}.get(name, i32)
+    return lib
+
+
+class QLoRAError(RuntimeError):
+    def __init__(self, code: int, where: str = ""):
+        self.code = code
+        super().__init__(f"{where}: {load().qlora_error_string(code).decode()} (code {code})")
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != 0:
+        raise QLoRAError(rc, where)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _need(t: torch.Tensor, dtype, name: str) -> None:
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous CUDA tensor of {dtype}, got {t.dtype} on {t.device}")
+
+
+# ---- host-only queries --------------------------------------------------------------------------
+
+def codebook():
+    """(levels float32[16], thresholds float32[15]) as the library uses them."""
+    lv = (ctypes.c_float * 16)()
+    th = (ctypes.c_float * 15)()
+    _check(load().qlora_nf4_codebook(lv, th), "qlora_nf4_codebook")
+    return np.array(lv, np.float32), np.array(th, np.float32)
+
+
+def storage_bytes(n: int) -> dict:
+    out = [ctypes.c_size_t() for _ in range(4)]
+    _check(load().qlora_nf4_storage_bytes(n, *[ctypes.byref(o) for o in out]), "qlora_nf4_storage_bytes")
+    return dict(codes=out[0].value, absmax=out[1].value, scale2=out[2].value, offset=out[3].value)
+
+
+def quantize_workspace_bytes(n: int) -> int:
+    b = ctypes.c_size_t()
+    _check(load().qlora_nf4_quantize_workspace(n, ctypes.byref(b)), "qlora_nf4_quantize_workspace")
+    return b.value
+
+
+def linear_workspace_bytes(T: int, N: int, K: int, r: int) -> int:
+    b = ctypes.c_size_t()
+    _check(load().qlora_linear_workspace(T, N, K, r, ctypes.byref(b)), "qlora_linear_workspace")
+    return b.value
+
+
+# ---- the NF4 tensor -----------------------------------------------------------------------------
+
+@dataclass
+class NF4Weight:
+    """Device buffers of an NF4 tensor with double-quantized constants (see qlora_nf4_tensor)."""
+    codes: torch.Tensor        # uint8 [ceil(n/2)]
+    absmax_e4m3: torch.Tensor  # uint8 [nb]
+    scale2: torch.Tensor       # float32 [ng]
+    offset: torch.Tensor       # float32 [1]
+    rows: int
+    cols: int
+
+    @classmethod
+    def empty(cls, rows: int, cols: int, device) -> "NF4Weight":
+        sb = storage_bytes(rows * cols)
+        u8 = dict(dtype=torch.uint8, device=device)
+        return cls(torch.empty(sb["codes"], **u8), torch.empty(sb["absmax"], **u8),
+                   torch.empty(sb["scale2"] // 4, dtype=torch.float32, device=device),
+                   torch.empty(1, dtype=torch.float32, device=device), rows, cols)
+
+    def struct(self) -> _NF4Struct:
+        return _NF4Struct(self.codes.data_ptr(), self.absmax_e4m3.data_ptr(), self.scale2.data_ptr(),
+                          self.offset.data_ptr(), self.rows, self.cols)
+
+    @property
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.codes, self.absmax_e4m3, self.scale2, self.offset))
+
+
+def quantize(w: torch.Tensor, out: NF4Weight | None = None, workspace: torch.Tensor | None = None,
+             stream=None) -> NF4Weight:
+    """NF4 + double quantization of a CUDA fp32 or bf16 tensor (1-D or 2-D, contiguous)."""
+    if w.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("quantize: w must be float32 or bfloat16")
+    _need(w, w.dtype, "w")
+    rows, cols = (w.shape[0], w.shape[1]) if w.dim() == 2 else (1, w.numel())
+    q = out if out is not None else NF4Weight.empty(rows, cols, w.device)
+    need = quantize_workspace_bytes(rows * cols)
+    ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=w.device)
+    st = q.struct()
+    _check(load().qlora_nf4_quantize(_ptr(w), QLORA_F32 if w.dtype == torch.float32 else QLORA_BF16, rows, cols,
+                                  ctypes.byref(st), _ptr(ws), ws.numel(), _stream(stream)), "qlora_nf4_quantize")
+    return q
+
+
+def dequantize(q: NF4Weight, dtype=torch.bfloat16, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    if dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("dequantize: dtype must be float32 or bfloat16")
+    o = out if out is not None else torch.empty(q.rows, q.cols, dtype=dtype, device=q.codes.device)
+    _need(o, dtype, "out")
+    st = q.struct()
+    _check(load().qlora_nf4_dequantize(ctypes.byref(st), _ptr(o), QLORA_F32 if dtype == torch.float32 else QLORA_BF16,
+                                    _stream(stream)), "qlora_nf4_dequantize")
+    return o
+
+
+def linear_fwd(X: torch.Tensor, q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,
+               save_u: bool = True, out: torch.Tensor | None = None, U_out: torch.Tensor | None = None,
+               workspace: torch.Tensor | None = None, stream=None):
+    """Y = X W~^T + (alpha/r) (X A^T) B^T.  Returns (Y, U) with U = (alpha/r) X A^T in bf16 (T x r) or None."""
+    T, K = X.shape
+    r = A.shape[0]
+    for t, n in ((X, "X"), (A, "A"), (B, "B")):
+        _need(t, torch.bfloat16, n)
+    Y = out if out is not None else torch.empty(T, q.rows, dtype=torch.bfloat16, device=X.device)
+    U = U_out if U_out is not None else (torch.empty(T, r, dtype=torch.bfloat16, device=X.device) if save_u else None)
+    ws = workspace if workspace is not None else torch.empty(linear_workspace_bytes(T, q.rows, q.cols, r),
+                                                             dtype=torch.uint8, device=X.device)
+    st = q.struct()
+    _check(load().qlora_linear_fwd(_ptr(X), T, ctypes.byref(st), _ptr(A), _ptr(B), r, float(alpha), _ptr(Y), _ptr(U),
+                                _ptr(ws), ws.numel(), _stream(stream)), "qlora_linear_fwd")
+    return Y, U
+
+
+def linear_bwd(dY: torch.Tensor, X: torch.Tensor, q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,
+               U: torch.Tensor | None = None, need_dx: bool = True, dX: torch.Tensor | None = None,
+               dA: torch.Tensor | None = None, dB: torch.Tensor | None = None,
+               workspace: torch.Tensor | None = None, stream=None):
+    """(dX bf16 or None, dA fp32 r x K, dB fp32 N x r); the frozen NF4 weight gets no gradient."""
+    T, K = X.shape
+    r = A.shape[0]
+    for t, n in ((dY, "dY"), (X, "X"), (A, "A"), (B, "B")):
+        _need(t, torch.bfloat16, n)
+    dev = X.device
+    dXo = dX if dX is not None else (torch.empty(T, K, dtype=torch.bfloat16, device=dev) if need_dx else None)
+    dAo = dA if dA is not None else torch.empty(r, K, dtype=torch.float32, device=dev)
+    dBo = dB if dB is not None else torch.empty(q.rows, r, dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else torch.empty(linear_workspace_bytes(T, q.rows, q.cols, r),
+                                                             dtype=torch.uint8, device=dev)
+    st = q.struct()
+    _check(load().qlora_linear_bwd(_ptr(dY), _ptr(X), T, ctypes.byref(st), _ptr(A), _ptr(B), r, float(alpha), _ptr(U),
+                                _ptr(dXo), _ptr(dAo), _ptr(dBo), _ptr(ws), ws.numel(), _stream(stream)),
+           "qlora_linear_bwd")
+    return dXo, dAo, dBo
+
+
+def get_status(stream=None) -> int:
+    """Synchronize the stream and return (and clear) the device status bits (STATUS_*)."""
+    v = ctypes.c_int()
+    rc = load().qlora_get_status(ctypes.byref(v), _stream(stream))
+    if rc not in (0, -6, -7):
+        _check(rc, "qlora_get_status")
+    return v.value
+
+
+def kernel_launches() -> int:
+    """Kernels launched by the library in this process so far."""
+    return int(load().qlora_kernel_launches())
+
+
+def profile_enable(on: bool = True) -> None:
+    _check(load().qlora_profile_enable(1 if on else 0), "qlora_profile_enable")
+
+
+def profile_read() -> dict:
+    """{kernel class: (launches, total device ms)} since the last read; clears the record."""
+    n = (ctypes.c_int64 * 5)()
+    ms = (ctypes.c_double * 5)()
+    _check(load().qlora_profile_read(n, ms), "qlora_profile_read")
+    return {name: (int(n[i]), float(ms[i])) for i, name in enumerate(PROF_NAMES)}

@@ -1,0 +1,487 @@
+// The library's C ABI (declared in include/qlora_nf4.h): argument checks, workspace layout, tensor-map
+// construction and kernel launches for the NF4 codec and the QLoRA linear layer. This is the only
+// translation unit with device code, so every kernel shares one status word per device.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "qlora_nf4.h"
+#include "codec.cuh"
+#include "gemm_sm100.cuh"
+
+namespace qnf4 {
+void build_nf4_codebook(float levels[16], float thresholds[15]);   // codebook.cpp
+
+namespace {
+
+constexpr int64_t kMaxNumel = int64_t(1) << 40;
+constexpr int64_t kMaxTokens = int64_t(65535) * 128;   // grid.y limit of the 128-row tiles
+constexpr int kTargetCtas = 2 * 148;                    // split heuristic: two waves of a B200
+std::atomic<int64_t> g_launches{0};
+inline int launched(int n = 1) {
+  g_launches.fetch_add(n, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+const CodebookArg& codebook() {
+  static CodebookArg cb;
+  static std::once_flag once;
+  std::call_once(once, [] { build_nf4_codebook(cb.levels, cb.thresholds); });
+  return cb;
+}
+
+// ---- device checks ------------------------------------------------------------------------------
+int check_device(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  int major = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  if (major != 10) return QLORA_ERR_UNSUPPORTED;
+  if (num_sms) *num_sms = sms;
+  return QLORA_OK;
+}
+
+// ---- profiling ----------------------------------------------------------------------------------
+struct ProfRec { int cls; cudaEvent_t a, b; };
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof;
+
+struct ProfScope {     // records an event pair around the launches in its lifetime
+  int cls; cudaStream_t st; cudaEvent_t a = nullptr, b = nullptr; bool on;
+  ProfScope(int c, cudaStream_t s) : cls(c), st(s) {
+    { std::lock_guard<std::mutex> g(g_prof_mu); on = g_prof_on; }
+    if (on && cudaEventCreate(&a) == cudaSuccess && cudaEventCreate(&b) == cudaSuccess) cudaEventRecord(a, st);
+    else on = false;
+  }
+  ~ProfScope() {
+    if (!on) return;
+    cudaEventRecord(b, st);
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    g_prof.push_back({cls, a, b});
+  }
+};
+
+// ---- tensor maps --------------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor: `inner` contiguous elements per row, `outer` rows, row pitch = inner elements.
+bool make_tmap(CUtensorMap* m, const void* ptr, bool bf16, uint64_t inner, uint64_t outer,
+               uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const uint64_t esz = bf16 ? 2 : 1;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * esz};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                        const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        bf16 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+// bf16 operand tiles: K-major tiles are {64 contraction, rows}; MN-major tiles are {64 MN, 64 contraction}.
+bool tmap_kmajor(CUtensorMap* m, const void* p, uint64_t contraction, uint64_t rows, uint32_t box_rows) {
+  return make_tmap(m, p, true, contraction, rows, 64, box_rows);
+}
+bool tmap_mnmajor(CUtensorMap* m, const void* p, uint64_t mn, uint64_t contraction) {
+  return make_tmap(m, p, true, mn, contraction, 64, 64);
+}
+
+// ---- GEMM launches ------------------------------------------------------------------------------
+template <class C>
+int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
+                const CUtensorMap& b2, const GemmParams& p, cudaStream_t st) {
+  auto kern = gemm_sm100_kernel<C>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, a2, b2, p, codebook());
+  return launched();
+}
+
+template <int BN> constexpr int skinny_stages() {
+  constexpr int stage = 128 * 64 * 2 + BN * 64 * 2;
+  return std::min(6, (200 * 1024) / stage);
+}
+
+struct Split { int splits, kb_split; };
+Split choose_split(int64_t tiles, int64_t nkb) {
+  int64_t want = std::max<int64_t>(1, cdiv(kTargetCtas, tiles));
+  want = std::min<int64_t>(want, std::max<int64_t>(1, nkb / 4));
+  const int64_t kb_split = cdiv(nkb, want);
+  return {static_cast<int>(cdiv(nkb, kb_split)), static_cast<int>(kb_split)};
+}
+
+enum class Skinny { kU, kV, kGrad };   // operand majors: (K,K), (K,MN), (MN,MN)
+
+// D[M][BN] partials = A (M x C) * B (BN x C)^T over contraction C, split along C.
+template <int BN, Skinny S>
+int launch_skinny(const CUtensorMap& a, const CUtensorMap& b, int64_t M, int64_t C, float* part,
+                  int64_t part_stride, cudaStream_t st) {
+  constexpr bool AMN = (S == Skinny::kGrad), BMN = (S != Skinny::kU);
+  using Cfg = GemmCfg<BN, AMN, BMN, BSrc::kTma, false, Epi::kF32Partial, skinny_stages<BN>()>;
+  const int64_t tiles = cdiv(M, 128), nkb = cdiv(C, 64);
+  const Split sp = choose_split(tiles, nkb);
+  GemmParams p{};
+  p.M = static_cast<int>(M); p.N = BN;
+  p.nkb_total = static_cast<int>(nkb); p.kb_split = sp.kb_split; p.nkb2 = 0;
+  p.out = part; p.ldo = BN; p.part_stride = part_stride;
+  return launch_gemm<Cfg>(dim3(1, static_cast<unsigned>(tiles), sp.splits), a, b, a, b, p, st);
+}
+template <Skinny S>
+int launch_skinny_bn(int bn, const CUtensorMap& a, const CUtensorMap& b, int64_t M, int64_t C, float* part,
+                     int64_t part_stride, cudaStream_t st) {
+  switch (bn) {
+    case 64: return launch_skinny<64, S>(a, b, M, C, part, part_stride, st);
+    case 128: return launch_skinny<128, S>(a, b, M, C, part, part_stride, st);
+    case 192: return launch_skinny<192, S>(a, b, M, C, part, part_stride, st);
+    case 256: return launch_skinny<256, S>(a, b, M, C, part, part_stride, st);
+  }
+  return QLORA_ERR_INVALID_ARG;
+}
+int64_t skinny_part_elems(int64_t M, int64_t C, int bn) {
+  const int64_t tiles = cdiv(M, 128);
+  const Split sp = choose_split(tiles, cdiv(C, 64));
+  return static_cast<int64_t>(sp.splits) * tiles * 128 * bn;
+}
+
+int reduce_after(const float* part, int64_t M, int64_t C, int R, int bn, float scale, void* out,
+                 Red mode, cudaStream_t st) {
+  const int64_t tiles = cdiv(M, 128);
+  const Split sp = choose_split(tiles, cdiv(C, 64));
+  const int64_t stride = tiles * 128 * bn;
+  const int64_t total = M * R;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(cdiv(total, 256), 148 * 16));
+  switch (mode) {
+    case Red::kRowsBf16:
+      split_reduce_kernel<Red::kRowsBf16><<<grid, 256, 0, st>>>(part, sp.splits, stride, bn, M, R, scale, out);
+      break;
+    case Red::kTransF32:
+      split_reduce_kernel<Red::kTransF32><<<grid, 256, 0, st>>>(part, sp.splits, stride, bn, M, R, scale, out);
+      break;
+    case Red::kRowsF32:
+      split_reduce_kernel<Red::kRowsF32><<<grid, 256, 0, st>>>(part, sp.splits, stride, bn, M, R, scale, out);
+      break;
+  }
+  return launched();
+}
+
+// ---- argument checks ----------------------------------------------------------------------------
+int check_nf4(const qlora_nf4_tensor* q) {
+  if (!q || !q->codes || !q->absmax_e4m3 || !q->scale2 || !q->offset) return QLORA_ERR_INVALID_ARG;
+  if (q->rows <= 0 || q->cols <= 0 || q->rows > kMaxNumel / q->cols) return QLORA_ERR_SHAPE;
+  if (!aligned16(q->codes) || !aligned16(q->absmax_e4m3) || !aligned16(q->scale2) || !aligned16(q->offset))
+    return QLORA_ERR_ALIGNMENT;
+  return QLORA_OK;
+}
+
+struct LinearWs { size_t sU, sV, part, total; };
+LinearWs linear_ws(int64_t T, int64_t N, int64_t K, int r) {
+  const int bn = static_cast<int>(cdiv(r, 64) * 64);
+  int64_t part = 0;
+  part = std::max(part, skinny_part_elems(T, K, bn));   // U
+  part = std::max(part, skinny_part_elems(T, N, bn));   // V
+  part = std::max(part, skinny_part_elems(K, T, bn));   // dA
+  part = std::max(part, skinny_part_elems(N, T, bn));   // dB
+  LinearWs w;
+  w.sU = 0;
+  w.sV = align256(static_cast<size_t>(T) * r * 2);
+  w.part = w.sV + align256(static_cast<size_t>(T) * r * 2);
+  w.total = w.part + align256(static_cast<size_t>(part) * 4);
+  return w;
+}
+
+int check_linear(const void* X, int64_t T, const qlora_nf4_tensor* W, const void* A, const void* B, int r,
+                 float alpha, void* ws, size_t ws_bytes) {
+  if (!X || !A || !B) return QLORA_ERR_INVALID_ARG;
+  if (int e = check_nf4(W)) return e;
+  if (r < 8 || r > 256 || r % 8 != 0 || !std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+  if (T < 1 || T > kMaxTokens || W->cols % 64 != 0 || W->rows % 8 != 0 || W->rows > (int64_t(1) << 30) ||
+      W->cols > (int64_t(1) << 30))
+    return QLORA_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(ws)) return QLORA_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < linear_ws(T, W->rows, W->cols, r).total) return QLORA_ERR_WORKSPACE;
+  return QLORA_OK;
+}
+
+// sU = s * X A^T (T x r, bf16) via the split adapter GEMM and its reduction.
+int compute_sU(const void* X, int64_t T, int64_t K, const void* A, int r, float s, void* sU, float* part,
+               cudaStream_t st) {
+  const int bn = static_cast<int>(cdiv(r, 64) * 64);
+  CUtensorMap ta, tb;
+  if (!tmap_kmajor(&ta, X, K, T, 128) || !tmap_kmajor(&tb, A, K, r, bn)) return QLORA_ERR_CUDA;
+  const int64_t stride = cdiv(T, 128) * 128 * bn;
+  if (int e = launch_skinny_bn<Skinny::kU>(bn, ta, tb, T, K, part, stride, st)) return e;
+  return reduce_after(part, T, K, r, bn, s, sU, Red::kRowsBf16, st);
+}
+
+}  // namespace
+}  // namespace qnf4
+
+using namespace qnf4;
+
+// ================================== C ABI ==========================================================
+extern "C" {
+
+int qlora_nf4_codebook(float* levels, float* thresholds) {
+  if (!levels || !thresholds) return QLORA_ERR_INVALID_ARG;
+  const CodebookArg& cb = codebook();
+  std::memcpy(levels, cb.levels, sizeof(cb.levels));
+  std::memcpy(thresholds, cb.thresholds, sizeof(cb.thresholds));
+  return QLORA_OK;
+}
+
+int qlora_nf4_storage_bytes(int64_t n, size_t* codes, size_t* absmax, size_t* scale2, size_t* offset) {
+  if (n <= 0 || n > kMaxNumel) return QLORA_ERR_SHAPE;
+  const int64_t nb = cdiv(n, kBlock), ng = cdiv(nb, kGroup);
+  if (codes) *codes = static_cast<size_t>(cdiv(n, 2));
+  if (absmax) *absmax = static_cast<size_t>(nb);
+  if (scale2) *scale2 = static_cast<size_t>(ng) * 4;
+  if (offset) *offset = 4;
+  return QLORA_OK;
+}
+
+int qlora_nf4_quantize_workspace(int64_t n, size_t* bytes) {
+  if (!bytes) return QLORA_ERR_INVALID_ARG;
+  if (n <= 0 || n > kMaxNumel) return QLORA_ERR_SHAPE;
+  const int64_t nb = cdiv(n, kBlock), ng = cdiv(nb, kGroup);
+  *bytes = align256(static_cast<size_t>(nb) * 4) + static_cast<size_t>(ng) * 8;
+  return QLORA_OK;
+}
+
+int qlora_nf4_quantize(const void* w, int w_dtype, int64_t rows, int64_t cols, const qlora_nf4_tensor* out,
+                       void* workspace, size_t workspace_bytes, qlora_stream_t stream) {
+  if (!w) return QLORA_ERR_INVALID_ARG;
+  if (w_dtype != QLORA_F32 && w_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
+  if (rows <= 0 || cols <= 0 || rows > kMaxNumel / cols) return QLORA_ERR_SHAPE;
+  if (int e = check_nf4(out)) return e;
+  if (out->rows != rows || out->cols != cols) return QLORA_ERR_SHAPE;
+  if (!aligned16(w) || !aligned16(workspace)) return QLORA_ERR_ALIGNMENT;
+  const int64_t n = rows * cols, nb = cdiv(n, kBlock), ng = cdiv(nb, kGroup);
+  size_t need = 0;
+  qlora_nf4_quantize_workspace(n, &need);
+  if (!workspace || workspace_bytes < need) return QLORA_ERR_WORKSPACE;
+  int sms = 0;
+  if (int e = check_device(&sms)) return e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float* c1 = static_cast<float*>(workspace);
+  double* gsum = reinterpret_cast<double*>(static_cast<char*>(workspace) + align256(static_cast<size_t>(nb) * 4));
+  ProfScope prof(QLORA_PROF_QUANTIZE, st);
+  const unsigned g1 = static_cast<unsigned>(std::min<int64_t>(ng, int64_t(sms) * 8));
+  if (w_dtype == QLORA_F32)
+    nf4_quantize_pass1<float><<<g1, kQuantThreads, 0, st>>>(static_cast<const float*>(w), n, out->codes, c1,
+                                                             gsum, ng, codebook());
+  else
+    nf4_quantize_pass1<__nv_bfloat16><<<g1, kQuantThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(w), n,
+                                                                     out->codes, c1, gsum, ng, codebook());
+  nf4_mean<<<1, kMeanThreads, 0, st>>>(gsum, ng, nb, out->offset);
+  nf4_dq_pass2<<<static_cast<unsigned>(cdiv(ng, 8)), 256, 0, st>>>(c1, nb, out->offset, out->absmax_e4m3,
+                                                                   out->scale2, ng);
+  return launched(3);
+}
+
+int qlora_nf4_dequantize(const qlora_nf4_tensor* q, void* out, int out_dtype, qlora_stream_t stream) {
+  if (!out) return QLORA_ERR_INVALID_ARG;
+  if (out_dtype != QLORA_F32 && out_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
+  if (int e = check_nf4(q)) return e;
+  if (!aligned16(out)) return QLORA_ERR_ALIGNMENT;
+  int sms = 0;
+  if (int e = check_device(&sms)) return e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t n = q->rows * q->cols;
+  const int64_t work = cdiv(n / 8, 256 * 4);
+  const unsigned grid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(work, int64_t(sms) * 8)));
+  ProfScope prof(QLORA_PROF_DEQUANTIZE, st);
+  if (out_dtype == QLORA_BF16)
+    nf4_dequantize_kernel<true><<<grid, 256, 0, st>>>(q->codes, q->absmax_e4m3, q->scale2, q->offset, n, out,
+                                                      codebook());
+  else
+    nf4_dequantize_kernel<false><<<grid, 256, 0, st>>>(q->codes, q->absmax_e4m3, q->scale2, q->offset, n, out,
+                                                       codebook());
+  return launched();
+}
+
+int qlora_linear_workspace(int64_t T, int64_t N, int64_t K, int r, size_t* bytes) {
+  if (!bytes) return QLORA_ERR_INVALID_ARG;
+  if (r < 8 || r > 256 || r % 8 != 0) return QLORA_ERR_INVALID_ARG;
+  if (T < 1 || T > kMaxTokens || N < 8 || K < 64 || N % 8 || K % 64) return QLORA_ERR_SHAPE;
+  *bytes = linear_ws(T, N, K, r).total;
+  return QLORA_OK;
+}
+
+int qlora_linear_fwd(const void* X, int64_t T, const qlora_nf4_tensor* W, const void* A, const void* B, int r,
+                     float alpha, void* Y, void* U_out, void* workspace, size_t workspace_bytes,
+                     qlora_stream_t stream) {
+  if (!Y) return QLORA_ERR_INVALID_ARG;
+  if (int e = check_linear(X, T, W, A, B, r, alpha, workspace, workspace_bytes)) return e;
+  if (!aligned16(Y) || !aligned16(U_out)) return QLORA_ERR_ALIGNMENT;
+  if (int e = check_device(nullptr)) return e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t N = W->rows, K = W->cols;
+  const float s = alpha / static_cast<float>(r);
+  const LinearWs L = linear_ws(T, N, K, r);
+  char* ws = static_cast<char*>(workspace);
+  void* sU = U_out ? U_out : ws + L.sU;
+  float* part = reinterpret_cast<float*>(ws + L.part);
+  {
+    ProfScope prof(QLORA_PROF_LORA, st);
+    if (int e = compute_sU(X, T, K, A, r, s, sU, part, st)) return e;
+  }
+  CUtensorMap tx, tc, tu, tb;
+  if (!tmap_kmajor(&tx, X, K, T, 128) || !make_tmap(&tc, W->codes, false, K / 2, N, 32, 256) ||
+      !tmap_kmajor(&tu, sU, r, T, 128) || !tmap_kmajor(&tb, B, r, N, 256))
+    return QLORA_ERR_CUDA;
+  using Cfg = GemmCfg<256, false, false, BSrc::kNf4, true, Epi::kBf16, 3>;
+  GemmParams p{};
+  p.M = static_cast<int>(T); p.N = static_cast<int>(N);
+  p.nkb_total = static_cast<int>(K / 64); p.kb_split = p.nkb_total; p.nkb2 = static_cast<int>(cdiv(r, 64));
+  p.e4m3 = W->absmax_e4m3; p.s2 = W->scale2; p.mu = W->offset; p.w_rows = N; p.w_cols = K;
+  p.out = Y; p.ldo = N;
+  ProfScope prof(QLORA_PROF_FWD_GEMM, st);
+  return launch_gemm<Cfg>(dim3(static_cast<unsigned>(cdiv(N, 256)), static_cast<unsigned>(cdiv(T, 128)), 1),
+                          tx, tc, tu, tb, p, st);
+}
+
+int qlora_linear_bwd(const void* dY, const void* X, int64_t T, const qlora_nf4_tensor* W, const void* A,
+                     const void* B, int r, float alpha, const void* U, void* dX, float* dA, float* dB,
+                     void* workspace, size_t workspace_bytes, qlora_stream_t stream) {
+  if (!dY || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if (int e = check_linear(X, T, W, A, B, r, alpha, workspace, workspace_bytes)) return e;
+  if (!aligned16(dY) || !aligned16(U) || !aligned16(dX) || !aligned16(dA) || !aligned16(dB))
+    return QLORA_ERR_ALIGNMENT;
+  if (int e = check_device(nullptr)) return e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t N = W->rows, K = W->cols;
+  const float s = alpha / static_cast<float>(r);
+  const int bn = static_cast<int>(cdiv(r, 64) * 64);
+  const LinearWs L = linear_ws(T, N, K, r);
+  char* ws = static_cast<char*>(workspace);
+  float* part = reinterpret_cast<float*>(ws + L.part);
+  void* sV = ws + L.sV;
+  const void* sU = U;
+  {
+    ProfScope prof(QLORA_PROF_LORA, st);
+    if (!sU) {
+      if (int e = compute_sU(X, T, K, A, r, s, ws + L.sU, part, st)) return e;
+      sU = ws + L.sU;
+    }
+    // sV = s * dY B  (T x r): contraction over the N output features; B is N x r, i.e. MN-major.
+    CUtensorMap tdy, tbl;
+    if (!tmap_kmajor(&tdy, dY, N, T, 128) || !tmap_mnmajor(&tbl, B, r, N)) return QLORA_ERR_CUDA;
+    if (int e = launch_skinny_bn<Skinny::kV>(bn, tdy, tbl, T, N, part, cdiv(T, 128) * 128 * bn, st)) return e;
+    if (int e = reduce_after(part, T, N, r, bn, s, sV, Red::kRowsBf16, st)) return e;
+  }
+  if (dX) {
+    CUtensorMap tdy, tc, tv, ta;
+    if (!tmap_kmajor(&tdy, dY, N, T, 128) || !make_tmap(&tc, W->codes, false, K / 2, N, 32, 64) ||
+        !tmap_kmajor(&tv, sV, r, T, 128) || !tmap_mnmajor(&ta, A, K, r))
+      return QLORA_ERR_CUDA;
+    using Cfg = GemmCfg<256, false, true, BSrc::kNf4, true, Epi::kBf16, 3>;
+    GemmParams p{};
+    p.M = static_cast<int>(T); p.N = static_cast<int>(K);
+    p.nkb_total = static_cast<int>(cdiv(N, 64)); p.kb_split = p.nkb_total; p.nkb2 = static_cast<int>(cdiv(r, 64));
+    p.e4m3 = W->absmax_e4m3; p.s2 = W->scale2; p.mu = W->offset; p.w_rows = N; p.w_cols = K;
+    p.out = dX; p.ldo = K;
+    ProfScope prof(QLORA_PROF_BWD_GEMM, st);
+    if (int e = launch_gemm<Cfg>(dim3(static_cast<unsigned>(cdiv(K, 256)), static_cast<unsigned>(cdiv(T, 128)), 1),
+                                 tdy, tc, tv, ta, p, st))
+      return e;
+  }
+  ProfScope prof(QLORA_PROF_LORA, st);
+  {
+    // dA^T[k][j] = sum_t X[t][k] sV[t][j]  -> dA (r x K), transposed in the reduction
+    CUtensorMap tx, tv;
+    if (!tmap_mnmajor(&tx, X, K, T) || !tmap_mnmajor(&tv, sV, r, T)) return QLORA_ERR_CUDA;
+    if (int e = launch_skinny_bn<Skinny::kGrad>(bn, tx, tv, K, T, part, cdiv(K, 128) * 128 * bn, st)) return e;
+    if (int e = reduce_after(part, K, T, r, bn, 1.0f, dA, Red::kTransF32, st)) return e;
+  }
+  {
+    // dB[n][j] = sum_t dY[t][n] sU[t][j]
+    CUtensorMap tdy, tu;
+    if (!tmap_mnmajor(&tdy, dY, N, T) || !tmap_mnmajor(&tu, sU, r, T)) return QLORA_ERR_CUDA;
+    if (int e = launch_skinny_bn<Skinny::kGrad>(bn, tdy, tu, N, T, part, cdiv(N, 128) * 128 * bn, st)) return e;
+    if (int e = reduce_after(part, N, T, r, bn, 1.0f, dB, Red::kRowsF32, st)) return e;
+  }
+  return QLORA_OK;
+}
+
+int qlora_get_status(int* device_status, qlora_stream_t stream) {
+  if (!device_status) return QLORA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return QLORA_ERR_CUDA;
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  *device_status = static_cast<int>(v);
+  if (v & kStatusTimeout) return QLORA_ERR_TIMEOUT;
+  if (v & kStatusNonfinite) return QLORA_ERR_NONFINITE;
+  return QLORA_OK;
+}
+
+const char* qlora_error_string(int code) {
+  switch (code) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_INVALID_ARG: return "invalid argument";
+    case QLORA_ERR_SHAPE: return "unsupported or inconsistent shape";
+    case QLORA_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+    case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    case QLORA_ERR_CUDA: return "CUDA call or kernel launch failed";
+    case QLORA_ERR_NONFINITE: return "non-finite value in a quantized input";
+    case QLORA_ERR_TIMEOUT: return "a kernel gave up waiting (bounded wait expired)";
+    case QLORA_ERR_UNSUPPORTED: return "device is not an sm_100 GPU";
+  }
+  return "unknown error code";
+}
+
+int qlora_profile_enable(int on) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  g_prof_on = (on != 0);
+  return QLORA_OK;
+}
+
+int qlora_profile_read(int64_t* launches, double* total_ms) {
+  if (!launches || !total_ms) return QLORA_ERR_INVALID_ARG;
+  std::vector<ProfRec> recs;
+  {
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    recs.swap(g_prof);
+  }
+  for (int i = 0; i < QLORA_PROF_COUNT; ++i) { launches[i] = 0; total_ms[i] = 0.0; }
+  int rc = QLORA_OK;
+  for (auto& r : recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess)
+      rc = QLORA_ERR_CUDA;
+    launches[r.cls] += 1;
+    total_ms[r.cls] += ms;
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  return rc;
+}
+
+int64_t qlora_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

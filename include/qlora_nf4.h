@@ -1,0 +1,198 @@
+/*
+ * qlora_nf4.h -- C ABI of the B200 (sm_100a) QLoRA NF4 library.
+ *
+ * The library implements one data path from the QLoRA pages: blockwise NF4 quantization of a frozen
+ * weight with double quantization of its block constants, dequantization, and the QLoRA linear layer
+ * (forward and backward) that consumes the quantized weight.
+ *
+ * Sources (pages by title and section):
+ *   [PEFT]  PEFT page, zerotofrontier.app/sft/peft:
+ *           "Block-wise quantization in one page", "NF4, derived from normal quantiles",
+ *           "Double quantization", "Paged optimizers, and QLoRA end to end", "The real way".
+ *   [EXPL]  QLoRA explainer, prism.theerrors.in ("QLoRA: Efficient Finetuning of Quantized LLMs"):
+ *           "For the curious", "Putting it together".
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers unless a parameter says "host". The caller owns and
+ *     allocates every buffer; the library never allocates device memory and keeps no per-call state.
+ *     Its only state is a constant-memory codebook and one status word per device.
+ *   - Every device pointer must be 16-byte aligned (QLORA_ERR_ALIGNMENT otherwise).
+ *   - Layouts are row-major and dense. bf16 tensors are passed as `const void*`/`void*`.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream) and return after enqueueing.
+ *     Argument checks happen on the host before anything is enqueued; a failed check enqueues nothing.
+ *   - Return value: QLORA_OK (0) or a negative QLORA_ERR_* code. Device-side conditions (non-finite
+ *     input, a bounded wait that gave up) are recorded in the device status word and reported by
+ *     qlora_get_status().
+ *   - Calls are reentrant and may run concurrently on different streams when their buffers
+ *     (including workspaces) do not overlap.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* qlora_stream_t;   /* a cudaStream_t */
+
+enum qlora_status_code {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = -1,  /* null pointer, bad dtype, bad rank r or alpha                     */
+  QLORA_ERR_SHAPE = -2,        /* a size that is <= 0, too large, or breaks a divisibility rule    */
+  QLORA_ERR_ALIGNMENT = -3,    /* a device pointer that is not 16-byte aligned                     */
+  QLORA_ERR_WORKSPACE = -4,    /* workspace missing or smaller than the matching *_workspace query  */
+  QLORA_ERR_CUDA = -5,         /* a CUDA runtime/driver call or kernel launch failed               */
+  QLORA_ERR_NONFINITE = -6,    /* (status) a quantized input held Inf or NaN                        */
+  QLORA_ERR_TIMEOUT = -7,      /* (status) a kernel's bounded wait gave up; its outputs are invalid */
+  QLORA_ERR_UNSUPPORTED = -8   /* the current device is not an sm_100 (B200-class) GPU             */
+};
+
+/* Bits of the device status word (qlora_get_status). */
+enum { QLORA_STATUS_NONFINITE = 1, QLORA_STATUS_TIMEOUT = 2 };
+
+/* Element types of quantize inputs and dequantize outputs. */
+enum { QLORA_F32 = 0, QLORA_BF16 = 1 };
+
+/*
+ * An NF4 tensor with double-quantized constants [PEFT "Double quantization"; EXPL "For the curious"].
+ * numel = rows * cols, flattened row-major; nb = ceil(numel/64) blocks; ng = ceil(nb/256) groups.
+ *   codes        ceil(numel/2) bytes; byte i = code(2i) << 4 | code(2i+1); for odd numel the last
+ *                low nibble is 0. Codes index the 16-level NF4 codebook [PEFT "NF4, ..."].
+ *   absmax_e4m3  nb bytes; E4M3 (OCP FP8) code of each block's mean-subtracted absmax constant.
+ *   scale2       ng floats; the fp32 second-level constant of each group of 256 blocks.
+ *   offset       1 float; the mean that was subtracted from the block constants.
+ * All four are device pointers owned by the caller; sizes come from qlora_nf4_storage_bytes().
+ */
+typedef struct qlora_nf4_tensor {
+  uint8_t* codes;
+  uint8_t* absmax_e4m3;
+  float* scale2;
+  float* offset;
+  int64_t rows;
+  int64_t cols;
+} qlora_nf4_tensor;
+
+/*
+ * The NF4 codebook [PEFT "NF4, derived from normal quantiles"]: 16 levels, 7 negative, an exact 0 at
+ * index 7, 8 positive, normal quantiles of evenly spaced probabilities from 0.9677 down to 0.5, rescaled
+ * so the ends are exactly -1 and +1; and the 15 decision thresholds (fp32-rounded midpoints of adjacent
+ * levels). An element w of a block with absmax a > 0 gets code #{j : w > thresholds[j] * a} in exact
+ * arithmetic (ties to the lower index); a block with a = 0 codes as 7.
+ * `levels` (16 floats) and `thresholds` (15 floats) are HOST arrays written by the call. Needs no GPU.
+ */
+int qlora_nf4_codebook(float* levels, float* thresholds);
+
+/*
+ * Exact byte sizes of the four arrays of an n-element NF4 tensor (host outputs; any may be NULL).
+ * Overhead of the constants: 8/64 + 32/(64*256) = 0.12695 bits per weight [PEFT "Double quantization"].
+ * Needs no GPU. QLORA_ERR_SHAPE if n <= 0 or n > 2^40.
+ */
+int qlora_nf4_storage_bytes(int64_t n, size_t* codes_bytes, size_t* absmax_bytes,
+                            size_t* scale2_bytes, size_t* offset_bytes);
+
+/* Device workspace bytes qlora_nf4_quantize needs for an n-element input (host output). No GPU. */
+int qlora_nf4_quantize_workspace(int64_t n, size_t* bytes);
+
+/*
+ * Quantize w (rows x cols, dtype QLORA_F32 or QLORA_BF16) into `out`, whose four pointers the caller
+ * has allocated with qlora_nf4_storage_bytes(rows*cols) and whose rows/cols must match
+ * [PEFT "Block-wise quantization in one page", "Double quantization"; EXPL "For the curious"]:
+ *   1. per block of 64 consecutive elements: absmax c1 (fp32), codes, two per byte;
+ *   2. mu = mean of all c1 (fp64 balanced pairwise tree over c1 zero-padded to max(256, 2^ceil(log2 nb))
+ *      leaves, divided by nb in fp64, rounded to fp32);
+ *   3. per group of 256 blocks: d = c1 - mu (fp32), s2 = max|d| / 448 (fp32), e = E4M3 round-to-nearest-
+ *      even, saturating, of d / s2 (e = 0 when s2 = 0).
+ * Any numel >= 1 is accepted; the last block and group may be partial. `workspace` (device, >=
+ * qlora_nf4_quantize_workspace bytes) holds the fp32 c1 and per-group partial sums between passes.
+ * A non-finite input sets QLORA_STATUS_NONFINITE; the outputs of that call are then unspecified.
+ * Results are deterministic and bit-identical run to run.
+ */
+int qlora_nf4_quantize(const void* w, int w_dtype, int64_t rows, int64_t cols,
+                       const qlora_nf4_tensor* out, void* workspace, size_t workspace_bytes,
+                       qlora_stream_t stream);
+
+/*
+ * Dequantize q into out (rows x cols, dtype QLORA_BF16 or QLORA_F32) [PEFT "Block-wise quantization in
+ * one page": look up the level and multiply back; "Double quantization"; EXPL "Putting it together":
+ * dequantized to bf16]:  c1_hat = fma(decode(e), s2, mu) (one fp32 rounding),
+ * w_hat = fp32(level[code] * c1_hat), then round-to-nearest-even bf16 for QLORA_BF16.
+ */
+int qlora_nf4_dequantize(const qlora_nf4_tensor* q, void* out, int out_dtype, qlora_stream_t stream);
+
+/*
+ * Device workspace bytes for qlora_linear_fwd / qlora_linear_bwd with T tokens, weight N x K (out x in)
+ * and LoRA rank r (host output). One buffer of this size serves both calls.
+ */
+int qlora_linear_workspace(int64_t T, int64_t N, int64_t K, int r, size_t* bytes);
+
+/*
+ * QLoRA linear forward [EXPL "Putting it together": Y = X dequant(W) + X L1 L2; PEFT "Paged optimizers,
+ * and QLoRA end to end": the frozen NF4 weight is dequantized to bf16 block by block, multiplied in
+ * 16-bit precision, and a bf16 LoRA adapter is added to the output]:
+ *     Y = X W~^T + s (X A^T) B^T,   s = alpha / r,   W~ = dequant(W) in bf16 (as qlora_nf4_dequantize).
+ *   X      T x K bf16          W  NF4 tensor, rows = N (out), cols = K (in)
+ *   A      r x K bf16          B  N x r bf16          Y  T x N bf16 (written)
+ *   U_out  T x r bf16 or NULL: if given, receives s * (X A^T) rounded to bf16, the scaled adapter
+ *          activation, in the form qlora_linear_bwd takes as U (saves recomputing it there).
+ * fp32 accumulation on the tensor cores. Rules: T >= 1; K % 64 == 0; N % 8 == 0; r % 8 == 0 and
+ * 8 <= r <= 256; alpha finite. `workspace` >= qlora_linear_workspace(T, N, K, r).
+ */
+int qlora_linear_fwd(const void* X, int64_t T, const qlora_nf4_tensor* W, const void* A,
+                     const void* B, int r, float alpha, void* Y, void* U_out, void* workspace,
+                     size_t workspace_bytes, qlora_stream_t stream);
+
+/*
+ * QLoRA linear backward [EXPL "Putting it together": gradients flow only into the adapters, never into
+ * the 4-bit weights; PEFT "Paged optimizers, and QLoRA end to end": gradients flow back through the
+ * dequantized weights to earlier layers]:
+ *     dX = dY W~ + s (dY B) A,   dA = s (dY B)^T X,   dB = s dY^T (X A^T);   no gradient for W.
+ *   dY  T x N bf16;  X, W, A, B, r, alpha as in qlora_linear_fwd;
+ *   U   T x r bf16 from qlora_linear_fwd's U_out with the same X, A, alpha, or NULL to recompute it;
+ *   dX  T x K bf16 or NULL (skip the input gradient, e.g. for the first layer);
+ *   dA  r x K fp32, dB  N x r fp32 (written, not accumulated; the adapters' gradients stay fp32).
+ * Same shape rules and workspace as qlora_linear_fwd.
+ */
+int qlora_linear_bwd(const void* dY, const void* X, int64_t T, const qlora_nf4_tensor* W,
+                     const void* A, const void* B, int r, float alpha, const void* U, void* dX,
+                     float* dA, float* dB, void* workspace, size_t workspace_bytes,
+                     qlora_stream_t stream);
+
+/*
+ * Synchronize `stream`, then read and clear the current device's status word into *device_status
+ * (host; a bitwise OR of QLORA_STATUS_* set by kernels since the last call). Returns QLORA_OK, or
+ * QLORA_ERR_NONFINITE / QLORA_ERR_TIMEOUT when the corresponding bit was set (TIMEOUT wins).
+ */
+int qlora_get_status(int* device_status, qlora_stream_t stream);
+
+/* Static English text for a QLORA_* code (never NULL). */
+const char* qlora_error_string(int code);
+
+/*
+ * Kernel timing for benchmarks. While enabled, the library records a CUDA event pair on the launch
+ * stream around every launch of its main matrix kernels and its codec kernels. qlora_profile_read
+ * synchronizes the recorded events and returns, per kernel class (QLORA_PROF_*), the number of launches
+ * and their summed device time in milliseconds (host arrays of QLORA_PROF_COUNT entries), then clears
+ * the record. Enabling does not change any result.
+ */
+enum {
+  QLORA_PROF_QUANTIZE = 0,    /* the three quantize kernels of one call, as one interval   */
+  QLORA_PROF_DEQUANTIZE = 1,
+  QLORA_PROF_FWD_GEMM = 2,    /* fused dequant + tensor-core forward (Y)                    */
+  QLORA_PROF_BWD_GEMM = 3,    /* fused dequant + tensor-core backward (dX)                  */
+  QLORA_PROF_LORA = 4,        /* the adapter kernels (U, V, dA, dB and their reductions)    */
+  QLORA_PROF_COUNT = 5
+};
+int qlora_profile_enable(int on);
+int qlora_profile_read(int64_t* launches, double* total_ms);
+
+/* Number of kernels the library has launched in this process (all devices, all streams). */
+int64_t qlora_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLORA_NF4_H */

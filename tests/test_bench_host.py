@@ -1,0 +1,63 @@
+"""Host-side logic of bench.py: the workload arithmetic, the roofline selection, and the multi-rank
+timing reduction (world size 2 over gloo on CPU)."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def test_flop_counts():
+    T, r = bench.TOKENS, bench.RANK_R
+    main = sum(2 * T * N * K for N, K in bench.SHAPES)
+    assert main == 2 * 8192 * (4096 * 4096 + 2 * 11008 * 4096)
+    assert bench.step_flops() == 2 * main + sum(6 * T * r * (N + K) for N, K in bench.SHAPES)
+    assert abs(bench.QUANT_B_PER_ELEM - 4.5159) < 1e-4 and abs(bench.DEQ_B_PER_ELEM - 2.5159) < 1e-4
+    assert bench.step_flops() / 16 < bench.oracle_sample_flops() < bench.step_flops() / 10
+
+
+def test_roofline_picks_the_dominant_class():
+    prof = {"quantize": (3, 0.5), "dequantize": (3, 0.2), "fwd_gemm": (3, 3.0), "bwd_gemm": (3, 3.5), "lora": (30, 0.4)}
+    peaks = {"hbm_gbs": 6543.1, "bf16_tflops": 1636.3, "bf16_tflops_sustained": 1375.0}
+    rf = bench.roofline(prof, 1, peaks, "measured")
+    assert rf["kernel"] == "bwd_gemm" and rf["bound"] == "tensor" and rf["peak"] == 1375.0
+    flops = sum(2 * bench.TOKENS * N * K + 2 * bench.TOKENS * bench.RANK_R * K for N, K in bench.SHAPES)
+    assert abs(rf["achieved"] - flops / 3.5e-3 / 1e12) < 0.01
+    assert abs(rf["frac"] - rf["achieved"] / 1375.0) < 1e-3
+    prof["quantize"] = (3, 9.0)
+    assert bench.roofline(prof, 1, peaks, "measured")["bound"] == "hbm"
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench.barrier()
+        got = bench.max_over_ranks(10.0 + 5.0 * rank)
+        q.put((rank, got, bench.dist_env()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[1] for r in res] == [15.0, 15.0]
+    assert [r[2][0] for r in res] == [0, 1] and all(r[2][2] == 2 for r in res)
+
+
+def test_single_process_reduction_is_identity():
+    assert bench.max_over_ranks(3.25) == 3.25

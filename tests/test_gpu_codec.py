@@ -1,0 +1,140 @@
+"""GPU parity of the NF4 codec against the oracle: codes, E4M3 constants, second-level scales, the mean
+and dequantized values must be bit-identical on the same seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def run_quantize(lib, w_np=None, w_t=None):
+    w = w_t if w_t is not None else torch.from_numpy(w_np).cuda()
+    q = lib.quantize(w)
+    st = lib.get_status()
+    return q, st
+
+
+def assert_same_as_oracle(q, ref):
+    n = ref.n
+    assert np.array_equal(q.codes.cpu().numpy(), ref.codes), "codes"
+    assert np.array_equal(q.absmax_e4m3.cpu().numpy(), ref.absmax_e4m3), "E4M3 constants"
+    assert np.array_equal(q.scale2.cpu().numpy().view(np.uint32), ref.scale2.view(np.uint32)), "scale2"
+    assert q.offset.cpu().numpy().view(np.uint32)[0] == np.float32(ref.offset).view(np.uint32), "mean"
+    assert q.codes.numel() == -(-n // 2)
+
+
+def assert_dequant_same(lib, q, ref, shape):
+    got16 = lib.dequantize(q, torch.bfloat16).cpu().view(torch.int16).numpy().view(np.uint16).reshape(-1)
+    assert np.array_equal(got16, O.dequantize(ref, "bf16").reshape(-1)), "bf16 dequant"
+    got32 = lib.dequantize(q, torch.float32).cpu().numpy().reshape(-1)
+    assert np.array_equal(got32.view(np.uint32), O.dequantize(ref, "f32").reshape(-1).view(np.uint32)), "fp32 dequant"
+
+
+def test_tiny_config_fp32(lib):
+    W = synth.weight_f32(256, 256, sigma=0.02, outlier_p=0.0, seed=0, tensor_id=1)
+    q, st = run_quantize(lib, W)
+    assert st == 0
+    ref = O.quantize(W)
+    assert_same_as_oracle(q, ref)
+    assert_dequant_same(lib, q, ref, W.shape)
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 63, 64, 65, 255, 257, 4097, 16383, 16384, 16385,
+                               3 * 16384 + 77, 100_003, 64 * 256 * 37 + 5])
+def test_ragged_sizes_fp32_and_bf16(lib, n):
+    x = synth.sweep_f32(n, seed=1, tensor_id=n % 1000)
+    q, st = run_quantize(lib, x.reshape(1, n))
+    assert st == 0
+    ref = O.quantize(x)
+    assert_same_as_oracle(q, ref)
+    assert_dequant_same(lib, q, ref, (1, n))
+    xb = synth.to_bf16(x)
+    qb, st = run_quantize(lib, w_t=xb.reshape(1, n).cuda())
+    refb = O.quantize(synth.bf16_bits(xb))
+    assert st == 0
+    assert_same_as_oracle(qb, refb)
+    qw, _ = run_quantize(lib, w_t=xb.float().reshape(1, n).cuda())   # bf16 input == its fp32 widening
+    assert torch.equal(qw.codes, qb.codes) and torch.equal(qw.absmax_e4m3, qb.absmax_e4m3)
+    assert torch.equal(qw.scale2, qb.scale2) and torch.equal(qw.offset, qb.offset)
+
+
+def test_many_groups_mean_tree(lib):
+    """ng = 1500 groups: the mean's fp64 tree spans several levels of the reduction kernel."""
+    n = 16384 * 1500 - 333
+    x = synth.sweep_f32(n, seed=2, tensor_id=5)
+    q, st = run_quantize(lib, x)
+    assert st == 0
+    ref = O.quantize(x)
+    assert_same_as_oracle(q, ref)
+
+
+def test_special_values(lib):
+    q_, T = O.nf4_codebook()
+    parts = [np.zeros(64 * 3, np.float32),                                  # all-zero blocks
+             np.full(64 * 256, 0.0173, np.float32),                         # equal constants: s2 = 0 group
+             (T.astype(np.float64) * 1.0).astype(np.float32),               # exact ties at a = 1
+             np.float32([1.0] + [-1.0] * 63),
+             np.float32([1e-40, -3e-39, 2e-45] + [0.0] * 61),               # subnormal block
+             np.float32([3e38, -1e38] + [1e30] * 62),                       # huge block
+             np.float32([-0.0] * 64),
+             synth.normal_f32(64 * 300 + 17, 0.02, 0, 31)]
+    x = np.concatenate(parts).astype(np.float32)
+    q, st = run_quantize(lib, x)
+    assert st == 0
+    ref = O.quantize(x)
+    assert_same_as_oracle(q, ref)
+    assert_dequant_same(lib, q, ref, x.shape)
+
+
+def test_constant_tensor_gives_zero_second_level_scale(lib):
+    x = np.full(64 * 512, -0.5, np.float32)
+    q, _ = run_quantize(lib, x)
+    ref = O.quantize(x)
+    assert_same_as_oracle(q, ref)
+    assert np.all(ref.scale2 == 0) and np.all(ref.absmax_e4m3 == 0)
+    assert_dequant_same(lib, q, ref, x.shape)
+
+
+@pytest.mark.parametrize("bad", [np.nan, np.inf, -np.inf])
+def test_nonfinite_input_sets_status(lib, bad):
+    x = synth.normal_f32(64 * 40, 0.02, 0, 41)
+    x[1000] = bad
+    lib.quantize(torch.from_numpy(x).cuda())
+    assert lib.get_status() & lib.STATUS_NONFINITE
+    assert lib.get_status() == 0          # reading clears it
+
+
+def test_full_size_7b_weight(lib):
+    """The 11008 x 4096 LLaMA-7B-shaped weight (N(0, 0.02^2) with 0.1 % x10 outliers), fp32 input."""
+    W = synth.weight_f32(11008, 4096, seed=0, tensor_id=1)
+    q, st = run_quantize(lib, W)
+    assert st == 0
+    ref = O.quantize(W)
+    assert_same_as_oracle(q, ref)
+    got = lib.dequantize(q, torch.bfloat16).cpu().view(torch.int16).numpy().view(np.uint16).reshape(-1)
+    assert np.array_equal(got, O.dequantize(ref, "bf16").reshape(-1))
+
+
+def test_sweep_size_sampled(lib):
+    """A 2^26-element sweep tensor: exact on every per-block quantity; dequant checked on a sample."""
+    n = 1 << 26
+    x = synth.sweep_f32(n, seed=0, tensor_id=3)
+    q, st = run_quantize(lib, x)
+    assert st == 0
+    ref = O.quantize(x)
+    assert_same_as_oracle(q, ref)
+    deq = lib.dequantize(q, torch.bfloat16).view(-1)
+    idx = torch.from_numpy(np.random.default_rng(0).integers(0, n, 200_000)).cuda()
+    got = deq[idx].cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, O.dequantize(ref, "bf16").reshape(-1)[idx.cpu().numpy()])
+
+
+def test_deterministic(lib):
+    x = synth.sweep_f32(1_000_003, seed=4, tensor_id=9)
+    a = lib.quantize(torch.from_numpy(x).cuda())
+    b = lib.quantize(torch.from_numpy(x).cuda())
+    for f in ("codes", "absmax_e4m3", "scale2", "offset"):
+        assert torch.equal(getattr(a, f), getattr(b, f))

@@ -1,0 +1,126 @@
+"""The C ABI without a GPU: the library loads, exports every declared entry point, builds the same
+codebook as the oracle (by an independent method), sizes buffers by the closed forms, and rejects bad
+arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def q():
+    from bit_nf4_quantized_14_b200 import build
+    build.build()
+    import bit_nf4_quantized_14_b200 as mod
+    return mod
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "qlora_nf4.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|int64_t|const char\*)\s+(qlora_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported(q):
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(q.lib, n), n
+
+
+def test_codebook_identical_to_oracle(q):
+    lv, th = q.codebook()
+    ql, qt = O.nf4_codebook()
+    assert np.array_equal(lv.view(np.uint32), ql.view(np.uint32))
+    assert np.array_equal(th.view(np.uint32), qt.view(np.uint32))
+
+
+@pytest.mark.parametrize("n", [1, 2, 63, 64, 65, 16383, 16384, 16385, 1 << 31, 65_000_000_000])
+def test_storage_bytes_closed_form(q, n):
+    assert q.storage_bytes(n) == O.storage_bytes(n)
+    nb, ng = -(-n // 64), -(-n // 16384)
+    assert q.quantize_workspace_bytes(n) >= 4 * nb + 8 * ng
+
+
+def test_workspace_queries_and_shape_rules(q):
+    assert q.linear_workspace_bytes(8192, 4096, 4096, 64) > 8192 * 64 * 2
+    for bad in [(0, 64, 64, 8), (16, 64, 100, 8), (16, 60, 64, 8)]:
+        with pytest.raises(q.QLoRAError) as e:
+            q.linear_workspace_bytes(*bad)
+        assert e.value.code == -2
+    for r in (0, 4, 12, 264):
+        with pytest.raises(q.QLoRAError) as e:
+            q.linear_workspace_bytes(16, 64, 64, r)
+        assert e.value.code == -1
+
+
+def _nf4(rows, cols, base=0x100000):
+    return q_struct(base, rows, cols)
+
+
+def q_struct(base, rows, cols):
+    import bit_nf4_quantized_14_b200 as mod
+    return mod._NF4Struct(base, base + 0x10000, base + 0x20000, base + 0x30000, rows, cols)
+
+
+V = ctypes.c_void_p
+
+
+def test_quantize_argument_errors_before_any_cuda_call(q):
+    L = q.lib
+    st = q_struct(0x100000, 4, 64)
+    ws = V(0x200000)
+    assert L.qlora_nf4_quantize(None, 0, 4, 64, ctypes.byref(st), ws, 1 << 20, None) == -1
+    assert L.qlora_nf4_quantize(V(0x300000), 7, 4, 64, ctypes.byref(st), ws, 1 << 20, None) == -1
+    assert L.qlora_nf4_quantize(V(0x300000), 0, 0, 64, ctypes.byref(st), ws, 1 << 20, None) == -2
+    assert L.qlora_nf4_quantize(V(0x300000), 0, 4, 65, ctypes.byref(st), ws, 1 << 20, None) == -2   # shape mismatch
+    assert L.qlora_nf4_quantize(V(0x300008), 0, 4, 64, ctypes.byref(st), ws, 1 << 20, None) == -3
+    assert L.qlora_nf4_quantize(V(0x300000), 0, 4, 64, ctypes.byref(st), ws, 8, None) == -4
+    assert L.qlora_nf4_quantize(V(0x300000), 0, 4, 64, None, ws, 1 << 20, None) == -1
+    bad = q_struct(0x100000, 4, 64)
+    bad.scale2 = 0x100004
+    assert L.qlora_nf4_quantize(V(0x300000), 0, 4, 64, ctypes.byref(bad), ws, 1 << 20, None) == -3
+
+
+def test_valid_call_without_a_gpu_reports_cuda_error_not_a_fallback(q):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("this box has a GPU")
+    st = q_struct(0x100000, 4, 64)
+    rc = q.lib.qlora_nf4_quantize(V(0x300000), 0, 4, 64, ctypes.byref(st), V(0x200000), 1 << 20, None)
+    assert rc in (-5, -8)
+    assert q.lib.qlora_nf4_dequantize(ctypes.byref(st), V(0x300000), 1, None) in (-5, -8)
+
+
+def test_linear_argument_errors(q):
+    L = q.lib
+    W = q_struct(0x100000, 64, 128)
+    X, A, B, Y, ws = V(0x300000), V(0x310000), V(0x320000), V(0x330000), V(0x400000)
+    big = 1 << 30
+    f = L.qlora_linear_fwd
+    assert f(None, 16, ctypes.byref(W), A, B, 8, 16.0, Y, None, ws, big, None) == -1
+    assert f(X, 16, ctypes.byref(W), A, B, 12, 16.0, Y, None, ws, big, None) == -1       # r % 8
+    assert f(X, 16, ctypes.byref(W), A, B, 8, float("nan"), Y, None, ws, big, None) == -1
+    assert f(X, 0, ctypes.byref(W), A, B, 8, 16.0, Y, None, ws, big, None) == -2
+    W2 = q_struct(0x100000, 64, 96)                                                        # K % 64
+    assert f(X, 16, ctypes.byref(W2), A, B, 8, 16.0, Y, None, ws, big, None) == -2
+    W3 = q_struct(0x100000, 60, 128)                                                       # N % 8
+    assert f(X, 16, ctypes.byref(W3), A, B, 8, 16.0, Y, None, ws, big, None) == -2
+    assert f(V(0x300002), 16, ctypes.byref(W), A, B, 8, 16.0, Y, None, ws, big, None) == -3
+    assert f(X, 16, ctypes.byref(W), A, B, 8, 16.0, Y, None, ws, 16, None) == -4
+    b = L.qlora_linear_bwd
+    assert b(X, X, 16, ctypes.byref(W), A, B, 8, 16.0, None, None, None, V(0x340000), ws, big, None) == -1
+    assert b(X, X, 16, ctypes.byref(W), A, B, 8, 16.0, V(0x350001), None, V(0x360000), V(0x370000), ws, big,
+             None) == -3
+
+
+def test_error_strings(q):
+    for c in range(-8, 1):
+        assert len(q.lib.qlora_error_string(c)) > 0
+    assert q.lib.qlora_error_string(-99) == b"unknown error code"
