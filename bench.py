@@ -26,7 +26,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -95,40 +94,62 @@ def barrier(device=None):
 # ---- clocks ---------------------------------------------------------------------------------------
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples the SM clock, its maximum, power and the active clock-event (throttle) reasons through
+    NVML every few milliseconds on a background thread while the timed region runs (read-only queries;
+    nothing about the GPU is changed)."""
+    REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+               "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+               "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+               "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+               "hw_power_brake_slowdown": "nvmlClocksEventReasonHwPowerBrakeSlowdown"}
 
-    def __init__(self, gpu_index: int):
-        self.idx, self.proc, self.lines = gpu_index, None, []
+    def __init__(self, torch_device_index: int, period_s: float = 0.005):
+        self.period, self.samples, self.stop_flag, self.thread, self.h = period_s, [], False, None, None
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            try:
+                import torch
+                uuid = str(torch.cuda.get_device_properties(torch_device_index).uuid)
+                self.h = nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self.h = nv.nvmlDeviceGetHandleByIndex(torch_device_index)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+        except Exception:
+            self.h = None
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_flag:
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetCurrentClocksEventReasons(self.h),
+                                     nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0))
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def start(self):
-        try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+        if self.h is None:
+            return
+        import threading
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
             return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        rows = [[c.strip() for c in ln.split(",")] for ln in out.strip().splitlines() if ln.count(",") >= 8]
-        if not rows:
+        self.stop_flag = True
+        self.thread.join(timeout=5)
+        if not self.samples:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        loaded = sorted(sm)[len(sm) // 2:] if sm else []
-        return {"sm_mhz": statistics.median(loaded) if loaded else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+        nv = self.nv
+        reasons = sorted({name for _, bits, _ in self.samples for name, attr in self.REASONS.items()
+                          if bits & getattr(nv, attr, 0)})
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples),
+                "power_w_max": round(max(s[2] for s in self.samples), 1), "source": "NVML, 5 ms period"}
 
 
 # ---- workload -------------------------------------------------------------------------------------
@@ -318,8 +339,7 @@ def run_gpu(args):
     # ---- device-resident timing ----
     q.profile_read()
     q.profile_enable(True)
-    clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[0])
-                          if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local_rank)
+    clocks = ClockSampler(local_rank)
     barrier(device)
     torch.cuda.synchronize()
     clocks.start()
@@ -341,6 +361,19 @@ def run_gpu(args):
     value = step_flops() * args.steps * world / (ms_max / 1e3) / 1e12
 
     # ---- end to end through the public API with pinned host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(q, wl, args, stream, device, world)
+    if rank == 0:
+        emit(args, world, ms_max, value, e2e, launches, prof, clk, status, wl)
+    if world > 1:
+        barrier(device)
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(q, wl, args, stream, device, world):
+    import torch
     host = []
     h2d = d2h = 0
     for d in wl:
@@ -374,50 +407,54 @@ def run_gpu(args):
     barrier(device)
     e_ms = max_over_ranks(e0.elapsed_time(e1), device)
     e2e_value = step_flops() * args.steps * world / (e_ms / 1e3) / 1e12
+    return {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms / args.steps, 3)}
 
-    if rank == 0:
-        peaks, kind = load_peaks()
-        nq = sum(N * K for N, K in SHAPES) * args.steps
-        parts = {}
-        for c, (n, t) in prof.items():
-            parts[c] = {"launches": n, "ms_total": round(t, 3)}
-        if prof["quantize"][1] > 0:
-            parts["quantize"]["GB/s"] = round(nq * QUANT_B_PER_ELEM / (prof["quantize"][1] / 1e3) / 1e9, 1)
-        if prof["dequantize"][1] > 0:
-            parts["dequantize"]["GB/s"] = round(nq * DEQ_B_PER_ELEM / (prof["dequantize"][1] / 1e3) / 1e9, 1)
-        for c, f in (("fwd_gemm", lambda N, K: 2 * TOKENS * N * K + 2 * TOKENS * RANK_R * N),
-                     ("bwd_gemm", lambda N, K: 2 * TOKENS * N * K + 2 * TOKENS * RANK_R * K)):
-            if prof[c][1] > 0:
-                parts[c]["TFLOP/s"] = round(sum(f(N, K) for N, K in SHAPES) * args.steps / (prof[c][1] / 1e3) / 1e12, 1)
-        line = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": WORKLOAD, "tokens": TOKENS, "r": RANK_R, "alpha": ALPHA,
-                           "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                           "l2": "no flush: each step reads ~1.1 GB of distinct inputs (fp32 weights, X, dY), "
-                                 "well above the 126 MB L2"},
-                "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                        "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms / args.steps, 3)},
-                "gpu_launches": int(launches),
-                "roofline": roofline(prof, args.steps, peaks, kind),
-                "clocks": clk, "parts": parts, "device_status": status}
-        if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline_line([d["host"] for d in wl])
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        barrier(device)
-        dist.destroy_process_group()
-    return 0
+
+def emit(args, world, ms_max, value, e2e, launches, prof, clk, status, wl):
+    peaks, kind = load_peaks()
+    nq = sum(N * K for N, K in SHAPES) * args.steps
+    parts = {}
+    for c, (n, t) in prof.items():
+        parts[c] = {"launches": n, "ms_total": round(t, 3)}
+    if prof["quantize"][1] > 0:
+        parts["quantize"]["GB/s"] = round(nq * QUANT_B_PER_ELEM / (prof["quantize"][1] / 1e3) / 1e9, 1)
+    if prof["dequantize"][1] > 0:
+        parts["dequantize"]["GB/s"] = round(nq * DEQ_B_PER_ELEM / (prof["dequantize"][1] / 1e3) / 1e9, 1)
+    for c, f in (("fwd_gemm", lambda N, K: 2 * TOKENS * N * K + 2 * TOKENS * RANK_R * N),
+                 ("bwd_gemm", lambda N, K: 2 * TOKENS * N * K + 2 * TOKENS * RANK_R * K)):
+        if prof[c][1] > 0:
+            parts[c]["TFLOP/s"] = round(sum(f(N, K) for N, K in SHAPES) * args.steps / (prof[c][1] / 1e3) / 1e12, 1)
+    line = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "tokens": TOKENS, "r": RANK_R, "alpha": ALPHA,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "no flush: each step reads ~1.1 GB of distinct inputs (fp32 weights, X, dY), "
+                             "well above the 126 MB L2"},
+            "e2e": e2e,
+            "gpu_launches": int(launches),
+            "roofline": roofline(prof, args.steps, peaks, kind),
+            "clocks": clk, "parts": parts, "device_status": status}
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_line([d["host"] for d in wl])
+    print(json.dumps(line), flush=True)
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) measurement")
+    ap.add_argument("--shapes", default="all",
+                    help="comma-separated NxK subset of the workload shapes (profiling runs), e.g. 4096x4096")
     args = ap.parse_args(argv)
+    if args.shapes != "all":
+        global SHAPES
+        SHAPES = [tuple(int(v) for v in sh.split("x")) for sh in args.shapes.split(",")]
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
