@@ -64,6 +64,7 @@ def _open() -> ctypes.CDLL:
         "qlora_nf4_storage_bytes": [i64, P(sz), P(sz), P(sz), P(sz)],
         "qlora_nf4_quantize_workspace": [i64, P(sz)],
         "qlora_nf4_quantize": [vp, i32, i64, i64, P(_NF4Struct), vp, sz, vp],
+        "qlora_nf4_quantize_noalloc": [vp, i32, i64, i64, P(_NF4Struct), vp],
         "qlora_nf4_dequantize": [P(_NF4Struct), vp, i32, vp],
         "qlora_linear_workspace": [i64, i64, i64, i32, P(sz)],
         "qlora_linear_fwd": [vp, i64, P(_NF4Struct), vp, vp, i32, ctypes.c_float, vp, vp, vp, sz, vp],
@@ -178,6 +179,24 @@ def quantize(w: torch.Tensor, out: NF4Weight | None = None, workspace: torch.Ten
     _check(load().qlora_nf4_quantize(_ptr(w), QLORA_F32 if w.dtype == torch.float32 else QLORA_BF16, rows, cols,
                                   ctypes.byref(st), _ptr(ws), ws.numel(), _stream(stream)), "qlora_nf4_quantize")
     return q
+
+
+NOALLOC_MAX_NUMEL = 1 << 26
+
+
+def quantize_noalloc(w: torch.Tensor, out: NF4Weight, stream=None) -> NF4Weight:
+    """qlora_nf4_quantize_noalloc: like quantize() but with the library's fixed internal scratch instead
+    of a workspace, for callers that cannot allocate device memory at the call (at most 2^26 elements;
+    calls that overlap on the GPU race on the shared scratch). `out` must be preallocated."""
+    if w.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("quantize_noalloc: w must be float32 or bfloat16")
+    _need(w, w.dtype, "w")
+    rows, cols = (w.shape[0], w.shape[1]) if w.dim() == 2 else (1, w.numel())
+    st = out.struct()
+    _check(load().qlora_nf4_quantize_noalloc(_ptr(w), QLORA_F32 if w.dtype == torch.float32 else QLORA_BF16,
+                                             rows, cols, ctypes.byref(st), _stream(stream)),
+           "qlora_nf4_quantize_noalloc")
+    return out
 
 
 def dequantize(q: NF4Weight, dtype=torch.bfloat16, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:

@@ -237,6 +237,38 @@ int compute_sU(const void* X, int64_t T, int64_t K, const void* A, int r, float 
   return reduce_after(part, T, K, r, bn, s, sU, Red::kRowsBf16, st);
 }
 
+// ---- fixed scratch of qlora_nf4_quantize_noalloc ---------------------------------------------------
+// The per-block constants (fp32, up to 2^20 of them) followed by the per-group fp64 sums (up to 4096).
+// In host code `g_noalloc_scratch` names a host-side stand-in, never the device array: its device
+// address is looked up once per device with cudaGetSymbolAddress and cached here.
+constexpr int64_t kNoallocBlocks = QLORA_NOALLOC_MAX_NUMEL / kBlock;
+constexpr int64_t kNoallocGroups = kNoallocBlocks / kGroup;
+constexpr size_t kNoallocC1Bytes = static_cast<size_t>(kNoallocBlocks) * 4;
+static_assert(kNoallocC1Bytes + static_cast<size_t>(kNoallocGroups) * 8 == QLORA_NOALLOC_SCRATCH_BYTES,
+              "scratch layout");
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_dev_ptr[kMaxDevices] = {};
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[QLORA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+// Device address of this device's scratch array (set-up on the first call per device).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return QLORA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> g(g_noalloc_mu);
+  if (!g_noalloc_dev_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return QLORA_ERR_CUDA;
+    g_noalloc_dev_ptr[dev] = p;
+  }
+  *out = g_noalloc_dev_ptr[dev];
+  return QLORA_OK;
+}
 }  // namespace
 }  // namespace qnf4
 
@@ -289,6 +321,36 @@ int qlora_nf4_quantize(const void* w, int w_dtype, int64_t rows, int64_t cols, c
   float* c1 = static_cast<float*>(workspace);
   double* gsum = reinterpret_cast<double*>(static_cast<char*>(workspace) + align256(static_cast<size_t>(nb) * 4));
   ProfScope prof(QLORA_PROF_QUANTIZE, st);
+  const unsigned g1 = static_cast<unsigned>(std::min<int64_t>(ng, int64_t(sms) * 8));
+  if (w_dtype == QLORA_F32)
+    nf4_quantize_pass1<float><<<g1, kQuantThreads, 0, st>>>(static_cast<const float*>(w), n, out->codes, c1,
+                                                             gsum, ng, codebook());
+  else
+    nf4_quantize_pass1<__nv_bfloat16><<<g1, kQuantThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(w), n,
+                                                                     out->codes, c1, gsum, ng, codebook());
+  nf4_mean<<<1, kMeanThreads, 0, st>>>(gsum, ng, nb, out->offset);
+  nf4_dq_pass2<<<static_cast<unsigned>(cdiv(ng, 8)), 256, 0, st>>>(c1, nb, out->offset, out->absmax_e4m3,
+                                                                   out->scale2, ng);
+  return launched(3);
+}
+
+int qlora_nf4_quantize_noalloc(const void* w, int w_dtype, int64_t rows, int64_t cols,
+                               const qlora_nf4_tensor* out, qlora_stream_t stream) {
+  if (!w) return QLORA_ERR_INVALID_ARG;
+  if (w_dtype != QLORA_F32 && w_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
+  if (rows <= 0 || cols <= 0 || rows > kMaxNumel / cols) return QLORA_ERR_SHAPE;
+  if (rows * cols > QLORA_NOALLOC_MAX_NUMEL) return QLORA_ERR_TOO_LARGE;
+  if (int e = check_nf4(out)) return e;
+  if (out->rows != rows || out->cols != cols) return QLORA_ERR_SHAPE;
+  if (!aligned16(w)) return QLORA_ERR_ALIGNMENT;
+  int sms = 0;
+  if (int e = check_device(&sms)) return e;
+  void* scratch = nullptr;
+  if (int e = noalloc_scratch(&scratch)) return e;
+  const int64_t n = rows * cols, nb = cdiv(n, kBlock), ng = cdiv(nb, kGroup);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float* c1 = static_cast<float*>(scratch);
+  double* gsum = reinterpret_cast<double*>(static_cast<char*>(scratch) + kNoallocC1Bytes);
   const unsigned g1 = static_cast<unsigned>(std::min<int64_t>(ng, int64_t(sms) * 8));
   if (w_dtype == QLORA_F32)
     nf4_quantize_pass1<float><<<g1, kQuantThreads, 0, st>>>(static_cast<const float*>(w), n, out->codes, c1,
@@ -451,6 +513,7 @@ const char* qlora_error_string(int code) {
     case QLORA_ERR_NONFINITE: return "non-finite value in a quantized input";
     case QLORA_ERR_TIMEOUT: return "a kernel gave up waiting (bounded wait expired)";
     case QLORA_ERR_UNSUPPORTED: return "device is not an sm_100 GPU";
+    case QLORA_ERR_TOO_LARGE: return "input exceeds the fixed scratch of the no-allocation quantize (2^26 elements)";
   }
   return "unknown error code";
 }

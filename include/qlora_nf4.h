@@ -48,7 +48,8 @@ enum qlora_status_code {
   QLORA_ERR_CUDA = -5,         /* a CUDA runtime/driver call or kernel launch failed               */
   QLORA_ERR_NONFINITE = -6,    /* (status) a quantized input held Inf or NaN                        */
   QLORA_ERR_TIMEOUT = -7,      /* (status) a kernel's bounded wait gave up; its outputs are invalid */
-  QLORA_ERR_UNSUPPORTED = -8   /* the current device is not an sm_100 (B200-class) GPU             */
+  QLORA_ERR_UNSUPPORTED = -8,  /* the current device is not an sm_100 (B200-class) GPU             */
+  QLORA_ERR_TOO_LARGE = -9     /* input larger than the fixed scratch of qlora_nf4_quantize_noalloc */
 };
 
 /* Bits of the device status word (qlora_get_status). */
@@ -114,6 +115,32 @@ int qlora_nf4_quantize_workspace(int64_t n, size_t* bytes);
 int qlora_nf4_quantize(const void* w, int w_dtype, int64_t rows, int64_t cols,
                        const qlora_nf4_tensor* out, void* workspace, size_t workspace_bytes,
                        qlora_stream_t stream);
+
+/*
+ * qlora_nf4_quantize without a caller-provided workspace. (The QLoRA pages have no counterpart; this is
+ * an interface variant of qlora_nf4_quantize, with identical results.)
+ *
+ * For callers that cannot allocate device memory at the point of the call: code running under a
+ * framework's caching allocator, where a cudaMalloc behind the framework's back can synchronize the
+ * device and fragment memory the framework manages; plugin or callback interfaces that hand over only
+ * the input and output buffers; and loops that forbid allocation after start-up. The caller still
+ * allocates `out` (qlora_nf4_storage_bytes); the intermediate per-block constants and per-group sums live
+ * in one fixed scratch array inside the library, QLORA_NOALLOC_SCRATCH_BYTES (about 4 MiB) of device
+ * memory that every GPU which loads the library holds until the process exits.
+ *   - rows * cols must not exceed QLORA_NOALLOC_MAX_NUMEL (2^26); larger inputs return
+ *     QLORA_ERR_TOO_LARGE and enqueue nothing.
+ *   - The first call on a device looks up that device's scratch address (host-side set-up, done once
+ *     per device); make that first call before any stream capture.
+ *   - Every call on a device shares the same scratch and nothing in it is cleared or kept between calls
+ *     (each call writes every scratch element it reads). Calls that can overlap on the GPU -- on
+ *     different streams without ordering between them -- race on the scratch and must not be issued.
+ *   - The call allocates nothing: no cudaMalloc/cudaFree and no allocating library routine.
+ * Other arguments, checks, status reporting and results are those of qlora_nf4_quantize.
+ */
+#define QLORA_NOALLOC_MAX_NUMEL (((int64_t)1) << 26)
+#define QLORA_NOALLOC_SCRATCH_BYTES ((size_t)4 * 1024 * 1024 + (size_t)8 * 4096)
+int qlora_nf4_quantize_noalloc(const void* w, int w_dtype, int64_t rows, int64_t cols,
+                               const qlora_nf4_tensor* out, qlora_stream_t stream);
 
 /*
  * Dequantize q into out (rows x cols, dtype QLORA_BF16 or QLORA_F32) [PEFT "Block-wise quantization in

@@ -121,6 +121,6 @@ def test_linear_argument_errors(q):
 
 
 def test_error_strings(q):
-    for c in range(-8, 1):
+    for c in range(-9, 1):
         assert len(q.lib.qlora_error_string(c)) > 0
     assert q.lib.qlora_error_string(-99) == b"unknown error code"
