@@ -11,6 +11,7 @@
 
 #include "qlora_nf4.h"
 #include "codec.cuh"
+#include "gemm_nf4w.cuh"
 #include "gemm_sm100.cuh"
 
 namespace qnf4 {
@@ -86,21 +87,29 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D row-major tensor: `inner` contiguous elements per row, `outer` rows, row pitch = inner elements.
-bool make_tmap(CUtensorMap* m, const void* ptr, bool bf16, uint64_t inner, uint64_t outer,
-               uint32_t box_inner, uint32_t box_outer) {
+// 2-D row-major tensor: `inner` contiguous elements per row, `outer` rows, row pitch = `pitch` elements.
+enum class TmType { kBf16, kU8, kF32 };
+bool make_tmap_t(CUtensorMap* m, const void* ptr, TmType t, uint64_t inner, uint64_t outer, uint64_t pitch,
+                 uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
   auto fn = encode_fn();
   if (!fn) return false;
-  const uint64_t esz = bf16 ? 2 : 1;
+  const uint64_t esz = t == TmType::kBf16 ? 2 : t == TmType::kU8 ? 1 : 4;
+  const CUtensorMapDataType dt = t == TmType::kBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                 : t == TmType::kU8  ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * esz};
+  cuuint64_t strides[1] = {pitch * esz};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
-                        const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        bf16 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+  const CUresult r = fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+bool make_tmap(CUtensorMap* m, const void* ptr, bool bf16, uint64_t inner, uint64_t outer,
+               uint32_t box_inner, uint32_t box_outer, bool swizzle128 = true) {
+  return make_tmap_t(m, ptr, bf16 ? TmType::kBf16 : TmType::kU8, inner, outer, inner, box_inner, box_outer,
+                     bf16 && swizzle128);
 }
 // bf16 operand tiles: K-major tiles are {64 contraction, rows}; MN-major tiles are {64 MN, 64 contraction}.
 bool tmap_kmajor(CUtensorMap* m, const void* p, uint64_t contraction, uint64_t rows, uint32_t box_rows) {
@@ -118,6 +127,55 @@ int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUt
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return QLORA_ERR_CUDA;
   kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, a2, b2, p, codebook());
+  return launched();
+}
+
+// Pitch (in blocks) of the expanded-constants buffer of a weight with K columns: a multiple of 4, so
+// the rows of the by-row layout are 16-byte aligned for TMA.
+inline int64_t scales_pitch(int64_t K) { return (K / 64 + 3) / 4 * 4; }
+
+// Fused weight GEMM of the linear layer (gemm_nf4w.cuh). act = X (fwd) or dY (bwd), T x Cn row-major;
+// lora_w = B (fwd, N x r) or A (bwd, r x K); uv = s U or s V (T x r); out = Y (T x N) or dX (T x K);
+// scales = workspace for the expanded block constants (N x scales_pitch(K) fp32).
+template <bool BWD>
+int launch_nf4_linear(const void* act, int64_t T, const qlora_nf4_tensor* W, const void* lora_w, int r,
+                      const void* uv, void* out, float* scales, cudaStream_t st) {
+  using Cfg = NF4WCfg<BWD, 2>;
+  const int64_t N = W->rows, K = W->cols, kb_w = K / 64;
+  const int64_t Cn = BWD ? N : K, F = BWD ? K : N;
+  int sms = 0;
+  if (int e = check_device(&sms)) return e;
+  // the stage-friendly fp32 constants: by column (kb_w rows of N) forward, by row (N rows) backward
+  const int64_t ld = BWD ? scales_pitch(K) : N;
+  const unsigned eg = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(cdiv(N * kb_w, 256), int64_t(sms) * 8)));
+  if (BWD)
+    nf4_expand_scales_kernel<false><<<eg, 256, 0, st>>>(W->absmax_e4m3, W->scale2, W->offset, N, kb_w, ld, scales);
+  else
+    nf4_expand_scales_kernel<true><<<eg, 256, 0, st>>>(W->absmax_e4m3, W->scale2, W->offset, N, kb_w, ld, scales);
+  if (int e = launched()) return e;
+  CUtensorMap tx, tc, tk, tuv, to;
+  bool ok = tmap_kmajor(&tx, act, Cn, T, 256) && tmap_kmajor(&tuv, uv, r, T, 256) &&
+            make_tmap(&to, out, true, F, T, 32, 16, false);
+  if (!BWD)
+    ok = ok && make_tmap(&tc, W->codes, false, K / 2, N, 32, 128) &&
+         make_tmap_t(&tk, scales, TmType::kF32, N, kb_w, N, 128, 1, false);
+  else
+    ok = ok && make_tmap(&tc, W->codes, false, K / 2, N, 64, 64) &&
+         make_tmap_t(&tk, scales, TmType::kF32, kb_w, N, ld, 4, 64, false);
+  if (!ok) return QLORA_ERR_CUDA;
+  NF4GemmParams p{};
+  p.T = static_cast<int>(T); p.F = static_cast<int>(F);
+  p.nkb = static_cast<int>(cdiv(Cn, 64)); p.nkb2 = static_cast<int>(cdiv(r, 64));
+  p.tiles_f = static_cast<int>(cdiv(F, 128));
+  p.num_tiles = static_cast<int>(p.tiles_f * cdiv(T, 256));
+  p.r = r;
+  p.w_rows = N; p.w_cols = K;
+  p.lora_w = static_cast<const __nv_bfloat16*>(lora_w);
+  auto kern = nf4_linear_gemm_kernel<Cfg>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(p.num_tiles, sms));
+  kern<<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, st>>>(tx, tc, tk, tuv, to, p, codebook());
   return launched();
 }
 
@@ -197,7 +255,7 @@ int check_nf4(const qlora_nf4_tensor* q) {
   return QLORA_OK;
 }
 
-struct LinearWs { size_t sU, sV, part, total; };
+struct LinearWs { size_t sU, sV, scales, part, total; };
 LinearWs linear_ws(int64_t T, int64_t N, int64_t K, int r) {
   const int bn = static_cast<int>(cdiv(r, 64) * 64);
   int64_t part = 0;
@@ -208,7 +266,8 @@ LinearWs linear_ws(int64_t T, int64_t N, int64_t K, int r) {
   LinearWs w;
   w.sU = 0;
   w.sV = align256(static_cast<size_t>(T) * r * 2);
-  w.part = w.sV + align256(static_cast<size_t>(T) * r * 2);
+  w.scales = w.sV + align256(static_cast<size_t>(T) * r * 2);
+  w.part = w.scales + align256(static_cast<size_t>(N) * scales_pitch(K) * 4);
   w.total = w.part + align256(static_cast<size_t>(part) * 4);
   return w;
 }
@@ -411,19 +470,8 @@ int qlora_linear_fwd(const void* X, int64_t T, const qlora_nf4_tensor* W, const 
     ProfScope prof(QLORA_PROF_LORA, st);
     if (int e = compute_sU(X, T, K, A, r, s, sU, part, st)) return e;
   }
-  CUtensorMap tx, tc, tu, tb;
-  if (!tmap_kmajor(&tx, X, K, T, 128) || !make_tmap(&tc, W->codes, false, K / 2, N, 32, 256) ||
-      !tmap_kmajor(&tu, sU, r, T, 128) || !tmap_kmajor(&tb, B, r, N, 256))
-    return QLORA_ERR_CUDA;
-  using Cfg = GemmCfg<256, false, false, BSrc::kNf4, true, Epi::kBf16, 3>;
-  GemmParams p{};
-  p.M = static_cast<int>(T); p.N = static_cast<int>(N);
-  p.nkb_total = static_cast<int>(K / 64); p.kb_split = p.nkb_total; p.nkb2 = static_cast<int>(cdiv(r, 64));
-  p.e4m3 = W->absmax_e4m3; p.s2 = W->scale2; p.mu = W->offset; p.w_rows = N; p.w_cols = K;
-  p.out = Y; p.ldo = N;
   ProfScope prof(QLORA_PROF_FWD_GEMM, st);
-  return launch_gemm<Cfg>(dim3(static_cast<unsigned>(cdiv(N, 256)), static_cast<unsigned>(cdiv(T, 128)), 1),
-                          tx, tc, tu, tb, p, st);
+  return launch_nf4_linear<false>(X, T, W, B, r, sU, Y, reinterpret_cast<float*>(ws + L.scales), st);
 }
 
 int qlora_linear_bwd(const void* dY, const void* X, int64_t T, const qlora_nf4_tensor* W, const void* A,
@@ -456,20 +504,8 @@ int qlora_linear_bwd(const void* dY, const void* X, int64_t T, const qlora_nf4_t
     if (int e = reduce_after(part, T, N, r, bn, s, sV, Red::kRowsBf16, st)) return e;
   }
   if (dX) {
-    CUtensorMap tdy, tc, tv, ta;
-    if (!tmap_kmajor(&tdy, dY, N, T, 128) || !make_tmap(&tc, W->codes, false, K / 2, N, 32, 64) ||
-        !tmap_kmajor(&tv, sV, r, T, 128) || !tmap_mnmajor(&ta, A, K, r))
-      return QLORA_ERR_CUDA;
-    using Cfg = GemmCfg<256, false, true, BSrc::kNf4, true, Epi::kBf16, 3>;
-    GemmParams p{};
-    p.M = static_cast<int>(T); p.N = static_cast<int>(K);
-    p.nkb_total = static_cast<int>(cdiv(N, 64)); p.kb_split = p.nkb_total; p.nkb2 = static_cast<int>(cdiv(r, 64));
-    p.e4m3 = W->absmax_e4m3; p.s2 = W->scale2; p.mu = W->offset; p.w_rows = N; p.w_cols = K;
-    p.out = dX; p.ldo = K;
     ProfScope prof(QLORA_PROF_BWD_GEMM, st);
-    if (int e = launch_gemm<Cfg>(dim3(static_cast<unsigned>(cdiv(K, 256)), static_cast<unsigned>(cdiv(T, 128)), 1),
-                                 tdy, tc, tv, ta, p, st))
-      return e;
+    if (int e = launch_nf4_linear<true>(dY, T, W, A, r, sV, dX, reinterpret_cast<float*>(ws + L.scales), st)) return e;
   }
   ProfScope prof(QLORA_PROF_LORA, st);
   {

@@ -335,4 +335,29 @@ __global__ void __launch_bounds__(256) nf4_dequantize_kernel(
   }
 }
 
+// Expand the double-quantized block constants of an NF4 weight (w_rows x w_cols, blocks of 64 along a
+// row) to fp32, c1_hat = fma(decode(e), s2, mu) -- the same single rounding as the dequantizer -- in the
+// layout the fused linear kernel loads one stage of at a time:
+//   by_column  out[kb * ld + n]  (one row per block column: a stage's 128 rows are contiguous)
+//   by_row     out[n * ld + kb]  (one row per weight row, ld a multiple of 4: a stage reads 4 columns)
+template <bool kByColumn>
+__global__ void __launch_bounds__(256) nf4_expand_scales_kernel(const uint8_t* __restrict__ e4m3,
+                                                                const float* __restrict__ s2,
+                                                                const float* __restrict__ mu_ptr,
+                                                                int64_t w_rows, int64_t kb_w, int64_t ld,
+                                                                float* __restrict__ out) {
+  const float mu = *mu_ptr;
+  const int64_t total = w_rows * kb_w;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    int64_t n, kb;
+    if constexpr (kByColumn) { kb = i / w_rows; n = i % w_rows; }   // writes coalesced along n
+    else { n = i / kb_w; kb = i % kb_w; }                           // reads and writes along kb
+    const int64_t blk = n * kb_w + kb;
+    const float c = __fmaf_rn(decode_e4m3(e4m3[blk]), s2[blk / kGroup], mu);
+    if constexpr (kByColumn) out[kb * ld + n] = c;
+    else out[n * ld + kb] = c;
+  }
+}
+
 }  // namespace qnf4

@@ -178,11 +178,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
 // Small helpers
 // ------------------------------------------------------------------------------------------------
 // Register-table lookup: every lane holds entry (lane & 15) of a 16-entry table; the result is entry
-// (idx & 15) of it. Only the low 4 bits of idx are used (16-lane segments), so idx needs no masking.
+// (idx & 15) of it. With 16-lane shuffle segments only the low 4 bits of idx select the source lane, so
+// idx needs no masking. The intrinsic is convergent, so the compiler keeps it where the whole warp runs.
 __device__ __forceinline__ float lut16(float table_reg, uint32_t idx) {
-  float r;
-  asm volatile("shfl.sync.idx.b32 %0, %1, %2, 0x101f, 0xffffffff;" : "=f"(r) : "f"(table_reg), "r"(idx));
-  return r;
+  return __shfl_sync(0xffffffffu, table_reg, static_cast<int>(idx), 16);
 }
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (lower address), .y = hi

@@ -122,3 +122,12 @@ def test_llama7b_shapes_sampled(lib, N, K):
     Vall = dY64 @ h["B"].astype(np.float64)
     assert rel(dA.cpu(), s * Vall.T @ X64) <= TOL
     assert rel(dB.cpu(), s * dY64.T @ (X64 @ h["A"].astype(np.float64).T)) <= TOL
+
+
+@pytest.mark.parametrize("N,K", [(4096, 256), (256, 4096)])
+def test_persistent_tiles_full_compare(lib, N, K):
+    """More output tiles than SMs (4096 features x 4096 tokens = 32 x 16 tiles, in the forward for the
+    first shape and in the backward for the second): each persistent CTA runs several tiles through the
+    shared-memory ring and both tensor-memory accumulators. Every output is compared."""
+    case = synth.linear_case(T=4096, N=N, K=K, r=64, alpha=16.0, seed=6)
+    run_and_check(lib, case)
