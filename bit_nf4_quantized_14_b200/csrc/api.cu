@@ -39,6 +39,68 @@ const CodebookArg& codebook() {
   return cb;
 }
 
+// The quantizer's bucket table: bucket b (1..31) covers t = w/a in [(b - 16.5)/15, (b - 15.5)/15],
+// widened by kBucketWiden for the approximate reciprocal; lo(b) counts the thresholds below it. Valid
+// only if every widened bucket holds at most one threshold (true for the NF4 thresholds, whose closest
+// pair is 0.0805 apart against a bucket width of 0.0667); checked here once.
+struct Buckets { BucketArg arg; bool ok; };
+const Buckets& buckets() {
+  static Buckets bk;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    const CodebookArg& cb = codebook();
+    bk.arg = BucketArg{};
+    bk.ok = true;
+    for (int b = 0; b < 32; ++b) {
+      const double jl = (b - 16.5) / 15.0 - kBucketWiden, ju = (b - 15.5) / 15.0 + kBucketWiden;
+      int lo = 0, inside = 0;
+      for (int j = 0; j < 15; ++j) {
+        const double t = cb.thresholds[j];
+        lo += (t < jl) ? 1 : 0;
+        inside += (t >= jl && t <= ju) ? 1 : 0;
+      }
+      if (inside > 1) bk.ok = false;
+      bk.arg.lo_nibbles[b / 8] |= static_cast<uint32_t>(lo) << (4 * (b % 8));
+    }
+  });
+  return bk;
+}
+
+// Launch with programmatic stream serialization: the kernel may start while its predecessor in the
+// stream drains, and waits for it (griddepcontrol.wait) before touching its results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// Workspace of the quantizer: per-block constants (fp32), per-slab tree sums (fp64), the mean pass's
+// per-CTA subtree sums (fp64) and its arrival counter; each part 256-byte aligned.
+struct QuantWs { size_t c1, ssum, partial, ticket, total; int64_t nslabs; unsigned mean_ctas; };
+QuantWs quant_ws(int64_t n) {
+  const int64_t nb = cdiv(n, kBlock), ns = cdiv(n, kSlabElems);
+  int64_t P = 1;
+  while (P < ns) P <<= 1;
+  QuantWs w;
+  w.nslabs = ns;
+  w.mean_ctas = static_cast<unsigned>(std::max<int64_t>(1, P / kTreeLeavesPerCta));
+  w.c1 = 0;
+  w.ssum = align256(static_cast<size_t>(nb) * 4);
+  w.partial = w.ssum + align256(static_cast<size_t>(ns) * 8);
+  w.ticket = w.partial + align256(static_cast<size_t>(w.mean_ctas) * 8);
+  w.total = w.ticket + 256;
+  return w;
+}
+
 // ---- device checks ------------------------------------------------------------------------------
 int check_device(int* num_sms) {
   int dev = 0;
@@ -297,14 +359,15 @@ int compute_sU(const void* X, int64_t T, int64_t K, const void* A, int r, float 
 }
 
 // ---- fixed scratch of qlora_nf4_quantize_noalloc ---------------------------------------------------
-// The per-block constants (fp32, up to 2^20 of them) followed by the per-group fp64 sums (up to 4096).
-// In host code `g_noalloc_scratch` names a host-side stand-in, never the device array: its device
-// address is looked up once per device with cudaGetSymbolAddress and cached here.
+// The quantizer's workspace (quant_ws) for the largest accepted input, 2^26 elements: 2^20 fp32
+// per-block constants, 2^14 fp64 slab sums, 8 fp64 subtree sums and the arrival counter. Smaller inputs
+// use a prefix of each part. In host code `g_noalloc_scratch` names a host-side stand-in, never the
+// device array: its device address is looked up once per device with cudaGetSymbolAddress and cached.
 constexpr int64_t kNoallocBlocks = QLORA_NOALLOC_MAX_NUMEL / kBlock;
-constexpr int64_t kNoallocGroups = kNoallocBlocks / kGroup;
+constexpr int64_t kNoallocSlabs = QLORA_NOALLOC_MAX_NUMEL / kSlabElems;
 constexpr size_t kNoallocC1Bytes = static_cast<size_t>(kNoallocBlocks) * 4;
-static_assert(kNoallocC1Bytes + static_cast<size_t>(kNoallocGroups) * 8 == QLORA_NOALLOC_SCRATCH_BYTES,
-              "scratch layout");
+constexpr size_t kNoallocSsumBytes = static_cast<size_t>(kNoallocSlabs) * 8;
+static_assert(kNoallocC1Bytes + kNoallocSsumBytes + 256 + 256 == QLORA_NOALLOC_SCRATCH_BYTES, "scratch layout");
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_dev_ptr[kMaxDevices] = {};
@@ -327,6 +390,39 @@ int noalloc_scratch(void** out) {
   }
   *out = g_noalloc_dev_ptr[dev];
   return QLORA_OK;
+}
+
+// Passes 1, 1b and 2 of the quantizer on stream st, workspace laid out by quant_ws(n).
+int run_quantize(const void* w, int w_dtype, int64_t n, const qlora_nf4_tensor* out, void* ws, cudaStream_t st) {
+  int sms = 0;
+  if (int e = check_device(&sms)) return e;
+  const Buckets& bk = buckets();
+  if (!bk.ok) return QLORA_ERR_UNSUPPORTED;
+  const QuantWs L = quant_ws(n);
+  char* base = static_cast<char*>(ws);
+  float* c1 = reinterpret_cast<float*>(base + L.c1);
+  double* ssum = reinterpret_cast<double*>(base + L.ssum);
+  double* partial = reinterpret_cast<double*>(base + L.partial);
+  unsigned* ticket = reinterpret_cast<unsigned*>(base + L.ticket);
+  const int64_t nb = cdiv(n, kBlock), ng = cdiv(nb, kGroup);
+  const unsigned g1 = static_cast<unsigned>(
+      std::min<int64_t>(cdiv(L.nslabs, kQuantThreads / 32), int64_t(sms) * kQuantMinBlocks));
+  if (w_dtype == QLORA_F32)
+    nf4_quantize_pass1<float><<<g1, kQuantThreads, 0, st>>>(static_cast<const float*>(w), n, out->codes, c1, ssum,
+                                                             L.nslabs, codebook(), bk.arg, ticket);
+  else
+    nf4_quantize_pass1<__nv_bfloat16><<<g1, kQuantThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(w), n,
+                                                                     out->codes, c1, ssum, L.nslabs, codebook(),
+                                                                     bk.arg, ticket);
+  if (int e = launched()) return e;
+  if (launch_pdl(nf4_mean, L.mean_ctas, kTreeThreads, st, ssum, L.nslabs, nb, partial, ticket, out->offset) !=
+      cudaSuccess)
+    return QLORA_ERR_CUDA;
+  if (int e = launched()) return e;
+  if (launch_pdl(nf4_dq_pass2, static_cast<unsigned>(cdiv(ng, 8)), 256u, st, c1, nb, out->offset,
+                 out->absmax_e4m3, out->scale2, ng) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return launched();
 }
 }  // namespace
 }  // namespace qnf4
@@ -357,8 +453,7 @@ int qlora_nf4_storage_bytes(int64_t n, size_t* codes, size_t* absmax, size_t* sc
 int qlora_nf4_quantize_workspace(int64_t n, size_t* bytes) {
   if (!bytes) return QLORA_ERR_INVALID_ARG;
   if (n <= 0 || n > kMaxNumel) return QLORA_ERR_SHAPE;
-  const int64_t nb = cdiv(n, kBlock), ng = cdiv(nb, kGroup);
-  *bytes = align256(static_cast<size_t>(nb) * 4) + static_cast<size_t>(ng) * 8;
+  *bytes = quant_ws(n).total;
   return QLORA_OK;
 }
 
@@ -370,27 +465,11 @@ int qlora_nf4_quantize(const void* w, int w_dtype, int64_t rows, int64_t cols, c
   if (int e = check_nf4(out)) return e;
   if (out->rows != rows || out->cols != cols) return QLORA_ERR_SHAPE;
   if (!aligned16(w) || !aligned16(workspace)) return QLORA_ERR_ALIGNMENT;
-  const int64_t n = rows * cols, nb = cdiv(n, kBlock), ng = cdiv(nb, kGroup);
-  size_t need = 0;
-  qlora_nf4_quantize_workspace(n, &need);
-  if (!workspace || workspace_bytes < need) return QLORA_ERR_WORKSPACE;
-  int sms = 0;
-  if (int e = check_device(&sms)) return e;
+  const int64_t n = rows * cols;
+  if (!workspace || workspace_bytes < quant_ws(n).total) return QLORA_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  float* c1 = static_cast<float*>(workspace);
-  double* gsum = reinterpret_cast<double*>(static_cast<char*>(workspace) + align256(static_cast<size_t>(nb) * 4));
   ProfScope prof(QLORA_PROF_QUANTIZE, st);
-  const unsigned g1 = static_cast<unsigned>(std::min<int64_t>(ng, int64_t(sms) * 8));
-  if (w_dtype == QLORA_F32)
-    nf4_quantize_pass1<float><<<g1, kQuantThreads, 0, st>>>(static_cast<const float*>(w), n, out->codes, c1,
-                                                             gsum, ng, codebook());
-  else
-    nf4_quantize_pass1<__nv_bfloat16><<<g1, kQuantThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(w), n,
-                                                                     out->codes, c1, gsum, ng, codebook());
-  nf4_mean<<<1, kMeanThreads, 0, st>>>(gsum, ng, nb, out->offset);
-  nf4_dq_pass2<<<static_cast<unsigned>(cdiv(ng, 8)), 256, 0, st>>>(c1, nb, out->offset, out->absmax_e4m3,
-                                                                   out->scale2, ng);
-  return launched(3);
+  return run_quantize(w, w_dtype, n, out, workspace, st);
 }
 
 int qlora_nf4_quantize_noalloc(const void* w, int w_dtype, int64_t rows, int64_t cols,
@@ -402,25 +481,10 @@ int qlora_nf4_quantize_noalloc(const void* w, int w_dtype, int64_t rows, int64_t
   if (int e = check_nf4(out)) return e;
   if (out->rows != rows || out->cols != cols) return QLORA_ERR_SHAPE;
   if (!aligned16(w)) return QLORA_ERR_ALIGNMENT;
-  int sms = 0;
-  if (int e = check_device(&sms)) return e;
+  if (int e = check_device(nullptr)) return e;
   void* scratch = nullptr;
   if (int e = noalloc_scratch(&scratch)) return e;
-  const int64_t n = rows * cols, nb = cdiv(n, kBlock), ng = cdiv(nb, kGroup);
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  float* c1 = static_cast<float*>(scratch);
-  double* gsum = reinterpret_cast<double*>(static_cast<char*>(scratch) + kNoallocC1Bytes);
-  const unsigned g1 = static_cast<unsigned>(std::min<int64_t>(ng, int64_t(sms) * 8));
-  if (w_dtype == QLORA_F32)
-    nf4_quantize_pass1<float><<<g1, kQuantThreads, 0, st>>>(static_cast<const float*>(w), n, out->codes, c1,
-                                                             gsum, ng, codebook());
-  else
-    nf4_quantize_pass1<__nv_bfloat16><<<g1, kQuantThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(w), n,
-                                                                     out->codes, c1, gsum, ng, codebook());
-  nf4_mean<<<1, kMeanThreads, 0, st>>>(gsum, ng, nb, out->offset);
-  nf4_dq_pass2<<<static_cast<unsigned>(cdiv(ng, 8)), 256, 0, st>>>(c1, nb, out->offset, out->absmax_e4m3,
-                                                                   out->scale2, ng);
-  return launched(3);
+  return run_quantize(w, w_dtype, rows * cols, out, scratch, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int qlora_nf4_dequantize(const qlora_nf4_tensor* q, void* out, int out_dtype, qlora_stream_t stream) {
@@ -432,15 +496,18 @@ int qlora_nf4_dequantize(const qlora_nf4_tensor* q, void* out, int out_dtype, ql
   if (int e = check_device(&sms)) return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t n = q->rows * q->cols;
-  const int64_t work = cdiv(n / 8, 256 * 4);
-  const unsigned grid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(work, int64_t(sms) * 8)));
+  const bool bf16 = out_dtype == QLORA_BF16;
+  auto kern = bf16 ? nf4_dequantize_kernel<true> : nf4_dequantize_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDeqSmemBytes) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDeqThreads, kDeqSmemBytes) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(
+      std::max<int64_t>(1, std::min<int64_t>(cdiv(n, kGroupElems), int64_t(sms) * std::max(per_sm, 1))));
   ProfScope prof(QLORA_PROF_DEQUANTIZE, st);
-  if (out_dtype == QLORA_BF16)
-    nf4_dequantize_kernel<true><<<grid, 256, 0, st>>>(q->codes, q->absmax_e4m3, q->scale2, q->offset, n, out,
-                                                      codebook());
-  else
-    nf4_dequantize_kernel<false><<<grid, 256, 0, st>>>(q->codes, q->absmax_e4m3, q->scale2, q->offset, n, out,
-                                                       codebook());
+  kern<<<grid, kDeqThreads, kDeqSmemBytes, st>>>(q->codes, q->absmax_e4m3, q->scale2, q->offset, n, out,
+                                                 codebook());
   return launched();
 }
 

@@ -3,10 +3,11 @@
 // Method (PEFT page, zerotofrontier.app/sft/peft, "Block-wise quantization in one page",
 // "NF4, derived from normal quantiles", "Double quantization", "The real way"; QLoRA explainer,
 // prism.theerrors.in, "For the curious"):
-//   pass 1  per block of 64 consecutive elements: absmax c1, 4-bit codes (two per byte), and per group
-//           of 256 blocks the fp64 balanced-tree sum of its c1 values;
-//   pass 1b the mean mu of all c1: the fp64 balanced tree continued over the group sums, / nb, -> fp32;
-//   pass 2  per group: d = c1 - mu, s2 = max|d| / 448, e = E4M3(d / s2) (round to nearest even, satfinite).
+//   pass 1  per block of 64 consecutive elements: absmax c1, 4-bit codes (two per byte), and per slab
+//           of 64 blocks the fp64 balanced-tree sum of its c1 values;
+//   pass 1b the mean mu of all c1: the fp64 balanced tree continued over the slab sums, / nb, -> fp32;
+//   pass 2  per group of 256 blocks: d = c1 - mu, s2 = max|d| / 448, e = E4M3(d / s2) (round to nearest
+//           even, satfinite).
 //   dequant c1_hat = fma(decode(e), s2, mu); w_hat = fp32(level[code] * c1_hat) -> bf16 (RNE) or fp32.
 //
 // Codes: the pages ask for the index of the nearest level. The library's rule is
@@ -14,7 +15,15 @@
 // exactly; ties go to the lower index; a block with a = 0 codes as 7. For fp32 w, T_j and a:
 //   w > T_j * a  <=>  w > RD(T_j * a)
 // where RD is the fp32 product rounded toward -inf (no fp32 value lies strictly between RD(P) and an
-// inexact P, subnormals included), so one __fmul_rd and one compare decide each threshold exactly.
+// inexact P, subnormals included), so one __fmul_rd and one compare decide a threshold exactly.
+//
+// Finding the one threshold to test. With t = w / a in [-1, 1], an fma with a magic constant puts the
+// integer b = 16 + round(15 * t') (t' = t up to a relative 2^-20 from the approximate reciprocal) into
+// the low five mantissa bits; bucket b spans 1/15 in t, less than the smallest gap between two
+// thresholds (0.0805), so it holds at most one threshold. A 32-entry table (one entry per lane) gives
+// lo(b), the number of thresholds certainly below t, and then code = lo + [w > RD(T_lo * a)] exactly.
+// The table is built and checked on the host (every bucket, widened by 2^-18, holds at most one
+// threshold); a block whose absmax is below 2^-120 is first scaled by 2^64 so the reciprocal stays finite.
 #pragma once
 
 #include <cuda_fp8.h>
@@ -28,196 +37,288 @@ struct CodebookArg {       // passed by value: lives in the kernel-parameter con
   float levels[16];
   float thresholds[15];
 };
+struct BucketArg {         // bucket b -> lo(b), 4 bits each
+  uint32_t lo_nibbles[4];
+};
 
 constexpr int kBlock = 64;          // first-level block (weights per absmax constant)
 constexpr int kGroup = 256;         // second-level block (constants per fp32 scale)
 constexpr int kGroupElems = kBlock * kGroup;
+constexpr int kSlabBlocks = 64;     // pass 1: one warp owns a slab of 64 blocks
+constexpr int kSlabElems = kSlabBlocks * kBlock;
+constexpr int kStepElems = 512;     // one warp step: 8 blocks, 16 elements per lane
 constexpr int kQuantThreads = 256;
+constexpr int kQuantMinBlocks = 3;
+constexpr float kBucketScale = 15.0f;
+constexpr float kBucketBias = 12582928.0f;   // 1.5 * 2^23 + 16
+constexpr double kBucketWiden = 0x1p-18;     // table margin in units of t
 
-// Code of w in a block with absmax a > 0. T points at the 15 thresholds in shared memory.
-__device__ __forceinline__ uint32_t nf4_code(float w, float a, const float* T, float t7) {
-  uint32_t c = (w > __fmul_rd(t7, a)) ? 8u : 0u;
-  c += (w > __fmul_rd(T[c + 3], a)) ? 4u : 0u;
-  c += (w > __fmul_rd(T[c + 1], a)) ? 2u : 0u;
-  c += (w > __fmul_rd(T[c], a)) ? 1u : 0u;
-  return c;
+__device__ __forceinline__ float rcp_approx(float x) {   // within 1 ulp, subnormal results kept
+  float r;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float fmax_nan(float a, float b) {   // NaN-propagating maximum
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
 }
 
-template <typename InT> struct QuantVec;
-template <> struct QuantVec<float> {          // 4 fp32 per 16-byte load, 16 lanes per block
-  static constexpr int kElems = 4;
-  __device__ static void widen(const uint4& v, float (&x)[4]) {
-    x[0] = __uint_as_float(v.x); x[1] = __uint_as_float(v.y);
-    x[2] = __uint_as_float(v.z); x[3] = __uint_as_float(v.w);
-  }
-  __device__ static float load1(const float* p) { return *p; }
+template <typename InT> struct Scalar;
+template <> struct Scalar<float> {
+  __device__ static float load(const float* p) { return *p; }
 };
-template <> struct QuantVec<__nv_bfloat16> {  // 8 bf16 per 16-byte load, 8 lanes per block
-  static constexpr int kElems = 8;
-  __device__ static void widen(const uint4& v, float (&x)[8]) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+template <> struct Scalar<__nv_bfloat16> {
+  __device__ static float load(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+};
+
+// One lane's 16 consecutive elements, kept as raw bits so the next step's loads can be in flight
+// while the current step computes.
+template <typename InT> struct Raw16;
+template <> struct Raw16<float> {
+  uint4 v[4];
+  __device__ void load(const float* p) {
+    const uint4* q = reinterpret_cast<const uint4*>(p);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      x[2 * i] = __uint_as_float(w[i] << 16);
-      x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    for (int k = 0; k < 4; ++k) v[k] = __ldcs(q + k);
+  }
+  __device__ void widen(float (&x)[16]) const {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      x[4 * k] = __uint_as_float(v[k].x); x[4 * k + 1] = __uint_as_float(v[k].y);
+      x[4 * k + 2] = __uint_as_float(v[k].z); x[4 * k + 3] = __uint_as_float(v[k].w);
     }
   }
-  __device__ static float load1(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+};
+template <> struct Raw16<__nv_bfloat16> {
+  uint4 v[2];
+  __device__ void load(const __nv_bfloat16* p) {
+    const uint4* q = reinterpret_cast<const uint4*>(p);
+    v[0] = __ldcs(q);
+    v[1] = __ldcs(q + 1);
+  }
+  __device__ void widen(float (&x)[16]) const {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint32_t u[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        x[8 * k + 2 * i] = __uint_as_float(u[i] << 16);
+        x[8 * k + 2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+      }
+    }
+  }
 };
 
-// fp64 balanced-tree sum of the 256 block constants of a group held in shared memory (one warp):
-// lane l sums leaves 8l..8l+7 as a balanced tree, then the 32 lane sums are combined pairwise.
-__device__ __forceinline__ double group_tree_sum(const float* c1s, int lane) {
-  double v[8];
+// Code of one element. lotab: lane b holds lo(b) (as raw bits); ttab: lane j holds T_j, lanes >= 15 +inf.
+template <bool kScaled>
+__device__ __forceinline__ uint32_t nf4_code(float x, float a, float sc, float r15, float lotab, float ttab) {
+  const float xs = kScaled ? x * sc : x;
+  const float z = __fmaf_rn(xs, r15, kBucketBias);
+  const uint32_t lo =
+      __float_as_uint(__shfl_sync(0xffffffffu, lotab, static_cast<int>(__float_as_uint(z))));
+  const float tl = __shfl_sync(0xffffffffu, ttab, static_cast<int>(lo));
+  return lo + ((x > __fmul_rd(tl, a)) ? 1u : 0u);
+}
+// Codes of 16 elements as 8 bytes, byte i = (code[2i] << 4) | code[2i+1] (even element high nibble).
+template <bool kScaled>
+__device__ __forceinline__ void nf4_codes16(const float (&x)[16], float a, float sc, float r15, float lotab,
+                                            float ttab, uint32_t& w0, uint32_t& w1) {
+  w0 = 0;
+  w1 = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = static_cast<double>(c1s[8 * lane + i]);
-  double s = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const double r = __shfl_down_sync(0xffffffffu, s, off);
-    if ((lane & (2 * off - 1)) == 0) s = s + r;   // left subtree + right subtree
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t hi = nf4_code<kScaled>(x[2 * i], a, sc, r15, lotab, ttab);
+    const uint32_t lo = nf4_code<kScaled>(x[2 * i + 1], a, sc, r15, lotab, ttab);
+    const uint32_t b = (hi << 4) | lo;
+    if (i < 4) w0 |= b << (8 * i);
+    else w1 |= b << (8 * (i - 4));
   }
-  return s;
 }
 
-// Pass 1. Grid-stride over groups of 256 blocks; 256 threads per CTA. Writes codes, c1 (fp32,
-// workspace) and the group's fp64 tree sum (workspace).
+// One step of a warp: lanes 4k..4k+3 hold block k's 64 elements (16 each). Returns the team's absmax
+// (NaN if the block holds a NaN); flags a non-finite block in `bad`.
+__device__ __forceinline__ float block_codes(const float (&x)[16], float lotab, float ttab, uint32_t& bad,
+                                             uint32_t& w0, uint32_t& w1) {
+  float m = fmax_nan(fmax_nan(fmax_nan(fabsf(x[0]), fabsf(x[1])), fmax_nan(fabsf(x[2]), fabsf(x[3]))),
+                     fmax_nan(fmax_nan(fabsf(x[4]), fabsf(x[5])), fmax_nan(fabsf(x[6]), fabsf(x[7]))));
+  m = fmax_nan(m, fmax_nan(fmax_nan(fmax_nan(fabsf(x[8]), fabsf(x[9])), fmax_nan(fabsf(x[10]), fabsf(x[11]))),
+                           fmax_nan(fmax_nan(fabsf(x[12]), fabsf(x[13])), fmax_nan(fabsf(x[14]), fabsf(x[15])))));
+  m = fmax_nan(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  m = fmax_nan(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  const float a = m;
+  bad |= (a <= 3.402823466e38f) ? 0u : 1u;        // false for NaN and +inf
+  const bool tiny = a < 0x1p-120f;
+  const float sc = tiny ? 0x1p64f : 1.0f;
+  const float r15 = kBucketScale * rcp_approx(a * sc);
+  if (__any_sync(0xffffffffu, tiny)) nf4_codes16<true>(x, a, sc, r15, lotab, ttab, w0, w1);
+  else nf4_codes16<false>(x, a, sc, r15, lotab, ttab, w0, w1);
+  if (!(a > 0.0f)) {                                // all-zero block (or NaN): code 7
+    w0 = 0x77777777u;
+    w1 = 0x77777777u;
+  }
+  return a;
+}
+
+// Pass 1. Each warp owns slabs gw, gw + nw, ... and walks them as a flat sequence of 8-block steps,
+// loading step i+1 while step i computes. Per slab it writes the 64 block constants (fp32) and their
+// fp64 balanced-tree sum. A ragged last slab is done by one warp at the end, with bounds on every element.
 template <typename InT>
-__global__ void __launch_bounds__(kQuantThreads) nf4_quantize_pass1(
+__global__ void __launch_bounds__(kQuantThreads, kQuantMinBlocks) nf4_quantize_pass1(
     const InT* __restrict__ w, int64_t n, uint8_t* __restrict__ codes, float* __restrict__ c1,
-    double* __restrict__ gsum, int64_t ngroups, CodebookArg cb) {
-  using V = QuantVec<InT>;
-  constexpr int E = V::kElems;                 // elements per thread per load
-  constexpr int LPB = kBlock / E;              // lanes per block
-  constexpr int LOADS = kGroupElems / E / kQuantThreads;  // 16-byte loads per thread per group
-  __shared__ float T[16];
-  __shared__ float c1s[kGroup];
-  const int tid = threadIdx.x, lane = tid & 31;
-  if (tid < 15) T[tid] = cb.thresholds[tid];
-  __syncthreads();
-  const float t7 = T[7];
+    double* __restrict__ ssum, int64_t nslabs, CodebookArg cb, BucketArg bk, unsigned* __restrict__ ticket) {
+  __shared__ float c1buf[kQuantThreads / 32][kSlabBlocks];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0u;    // arrival counter of the mean pass
+  const float lotab = __uint_as_float((bk.lo_nibbles[lane >> 3] >> (4 * (lane & 7))) & 0xFu);
+  const float ttab = (lane < 15) ? cb.thresholds[lane] : __int_as_float(0x7F800000);
+  const int64_t nb = (n + kBlock - 1) / kBlock;
+  const int64_t nfull = n / kSlabElems;
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * (kQuantThreads / 32) + warp;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * (kQuantThreads / 32);
+  float* cb_w = c1buf[warp];
+  uint32_t bad = 0;
 
-  for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
-    const int64_t gbase = g * kGroupElems;
-    const bool full = gbase + kGroupElems <= n;
-    if (full) {
-      uint4 v[LOADS];
-      const uint4* src = reinterpret_cast<const uint4*>(w + gbase);
+  auto finish_slab = [&](int64_t s) {      // constants out, and the slab's 64-leaf fp64 tree
+    __syncwarp();
+    const float l0 = cb_w[2 * lane], l1 = cb_w[2 * lane + 1];
+    const int64_t gb = s * kSlabBlocks + 2 * lane;
+    if (gb + 1 < nb) *reinterpret_cast<float2*>(c1 + gb) = make_float2(l0, l1);
+    else if (gb < nb) c1[gb] = l0;
+    double t = static_cast<double>(l0) + static_cast<double>(l1);
 #pragma unroll
-      for (int i = 0; i < LOADS; ++i) v[i] = __ldcs(src + tid + kQuantThreads * i);
-#pragma unroll
-      for (int i = 0; i < LOADS; ++i) {
-        float x[E];
-        V::widen(v[i], x);
-        uint32_t m = 0;
-#pragma unroll
-        for (int e = 0; e < E; ++e) m = max(m, __float_as_uint(x[e]) & 0x7FFFFFFFu);
-#pragma unroll
-        for (int off = LPB / 2; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
-        const int blk = (tid + kQuantThreads * i) / LPB;  // block index within the group
-        if (m >= 0x7F800000u) {
-          if ((lane % LPB) == 0) raise_status(kStatusNonfinite);
-        }
-        const float a = __uint_as_float(m);
-        uint32_t packed = 0;
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const uint32_t c = (a > 0.0f) ? nf4_code(x[e], a, T, t7) : 7u;
-          // byte e/2 of this thread's code bytes: even element high nibble, odd element low nibble
-          packed |= c << (8 * (e >> 1) + ((e & 1) ? 0 : 4));
-        }
-        const int64_t ebase = gbase + static_cast<int64_t>(E) * (tid + kQuantThreads * i);
-        if constexpr (E == 4) {
-          *reinterpret_cast<uint16_t*>(codes + ebase / 2) = static_cast<uint16_t>(packed);
-        } else {
-          *reinterpret_cast<uint32_t*>(codes + ebase / 2) = packed;
-        }
-        if ((lane % LPB) == 0) c1s[blk] = a;
-      }
-    } else {
-      // Ragged last group: scalar loads, one block per LPB-lane team, bounds on every element.
-      for (int blk = tid / LPB; blk < kGroup; blk += kQuantThreads / LPB) {
-        const int64_t b0 = gbase + static_cast<int64_t>(blk) * kBlock;
-        float x[E];
-        uint32_t m = 0;
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const int64_t idx = b0 + (lane % LPB) * E + e;
-          x[e] = (idx < n) ? V::load1(w + idx) : 0.0f;
-          m = max(m, __float_as_uint(x[e]) & 0x7FFFFFFFu);
-        }
-#pragma unroll
-        for (int off = LPB / 2; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
-        if (m >= 0x7F800000u && (lane % LPB) == 0) raise_status(kStatusNonfinite);
-        const float a = __uint_as_float(m);
-#pragma unroll
-        for (int e = 0; e < E; e += 2) {
-          const int64_t idx = b0 + (lane % LPB) * E + e;
-          if (idx < n) {
-            const uint32_t hi = (a > 0.0f) ? nf4_code(x[e], a, T, t7) : 7u;
-            const uint32_t lo = (idx + 1 < n) ? ((a > 0.0f) ? nf4_code(x[e + 1], a, T, t7) : 7u) : 0u;
-            codes[idx / 2] = static_cast<uint8_t>((hi << 4) | lo);
-          }
-        }
-        if ((lane % LPB) == 0) c1s[blk] = (b0 < n) ? a : 0.0f;
-      }
+    for (int off = 1; off < 32; off <<= 1) {
+      const double r = __shfl_down_sync(0xffffffffu, t, off);
+      if ((lane & (2 * off - 1)) == 0) t = t + r;    // left subtree + right subtree
     }
-    __syncthreads();
-    const int64_t nb = (n + kBlock - 1) / kBlock;
-    for (int b = tid; b < kGroup; b += kQuantThreads) {
-      const int64_t gb = g * kGroup + b;
-      if (gb < nb) c1[gb] = c1s[b];
-    }
-    if (tid < 32) {
-      const double s = group_tree_sum(c1s, lane);
-      if (lane == 0) gsum[g] = s;
-    }
-    __syncthreads();
+    if (lane == 0) ssum[s] = t;
+    __syncwarp();
+  };
+
+  const int64_t my_slabs = (gw < nfull) ? (nfull - 1 - gw) / nw + 1 : 0;
+  const int64_t steps = my_slabs * (kSlabElems / kStepElems);
+  Raw16<InT> cur, nxt;
+  if (steps > 0) nxt.load(w + gw * kSlabElems + 16 * lane);
+  for (int64_t i = 0; i < steps; ++i) {
+    const int64_t s = gw + (i >> 3) * nw;
+    const int it = static_cast<int>(i & 7);
+    cur = nxt;
+    if (i + 1 < steps)
+      nxt.load(w + (gw + ((i + 1) >> 3) * nw) * kSlabElems + ((i + 1) & 7) * kStepElems + 16 * lane);
+    float x[16];
+    cur.widen(x);
+    const int64_t e0 = s * kSlabElems + it * kStepElems + 16 * lane;
+    uint32_t w0, w1;
+    const float a = block_codes(x, lotab, ttab, bad, w0, w1);
+    *reinterpret_cast<uint2*>(codes + (e0 >> 1)) = make_uint2(w0, w1);
+    if ((lane & 3) == 0) cb_w[it * 8 + (lane >> 2)] = a;
+    if (it == 7) finish_slab(s);
   }
+  if (nfull < nslabs && gw == nfull % nw) {          // the ragged last slab
+    const int64_t s = nfull;
+    for (int it = 0; it < kSlabElems / kStepElems; ++it) {
+      const int64_t e0 = s * kSlabElems + it * kStepElems + 16 * lane;
+      float x[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) x[e] = (e0 + e < n) ? Scalar<InT>::load(w + e0 + e) : 0.0f;
+      uint32_t w0, w1;
+      const float a = block_codes(x, lotab, ttab, bad, w0, w1);
+      for (int b = 0; b < 8; ++b) {
+        const int64_t idx = e0 + 2 * b;
+        if (idx < n) {
+          uint32_t byte = ((b < 4 ? w0 : w1) >> (8 * (b & 3))) & 0xFFu;
+          if (idx + 1 >= n) byte &= 0xF0u;                     // odd n: the final low nibble is 0
+          codes[idx >> 1] = static_cast<uint8_t>(byte);
+        }
+      }
+      if ((lane & 3) == 0) cb_w[it * 8 + (lane >> 2)] = a;
+    }
+    finish_slab(s);
+  }
+  if (bad) raise_status(kStatusNonfinite);
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// Pass 1b. One CTA: the fp64 balanced tree over the group sums zero-padded to P = 2^ceil(log2 ng)
-// leaves, continued to the root; mu = fp32(fp64(S / nb)).
-constexpr int kMeanThreads = 1024;
-__global__ void __launch_bounds__(kMeanThreads) nf4_mean(const double* __restrict__ gsum,
-                                                        int64_t ngroups, int64_t nblocks,
-                                                        float* __restrict__ mu_out) {
-  __shared__ double s[kMeanThreads];
+// Pass 1b. The fp64 balanced tree over the slab sums zero-padded to P = 2^ceil(log2 ns) leaves (the
+// same value as the tree over all block constants padded with zeros: zero subtrees add exactly 0).
+// CTA q reduces the aligned subtree of P / gridDim.x <= 2048 leaves; the last CTA to arrive combines
+// the gridDim.x subtree sums (a power of two) and writes mu = fp32(S / nb).
+constexpr int kTreeThreads = 256;
+constexpr int kTreeLeavesPerCta = 8 * kTreeThreads;
+__device__ __forceinline__ double cta_tree(double v, int nvals, double* sh) {
+  sh[threadIdx.x] = v;
+  __syncthreads();
+  for (int len = nvals / 2; len >= 1; len >>= 1) {
+    double x = 0.0;
+    if (static_cast<int>(threadIdx.x) < len) x = sh[2 * threadIdx.x] + sh[2 * threadIdx.x + 1];
+    __syncthreads();
+    if (static_cast<int>(threadIdx.x) < len) sh[threadIdx.x] = x;
+    __syncthreads();
+  }
+  return sh[0];
+}
+__global__ void __launch_bounds__(kTreeThreads) nf4_mean(const double* __restrict__ ssum, int64_t ns,
+                                                        int64_t nb, double* __restrict__ partial,
+                                                        unsigned* __restrict__ ticket, float* __restrict__ mu_out) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ double sh[kTreeThreads];
+  __shared__ int is_last;
   int64_t P = 1;
-  while (P < ngroups) P <<= 1;
-  const int nthreads = static_cast<int>(P < kMeanThreads ? P : kMeanThreads);
-  const int64_t chunk = P / nthreads;            // a power of two
-  const int tid = threadIdx.x;
+  while (P < ns) P <<= 1;
+  const int64_t L = P / gridDim.x;
+  const int per = static_cast<int>(L > kTreeThreads ? L / kTreeThreads : 1);   // 1, 2, 4 or 8
+  const int nv = static_cast<int>(L > kTreeThreads ? kTreeThreads : L);
   double v = 0.0;
-  if (tid < nthreads) {
-    // serial balanced tree over leaves [tid*chunk, (tid+1)*chunk): a binary counter of subtrees
-    double stack[48];
-    int top_level = 0;
-    for (int64_t i = 0; i < chunk; ++i) {
-      const int64_t idx = static_cast<int64_t>(tid) * chunk + i;
-      double x = (idx < ngroups) ? gsum[idx] : 0.0;
-      int64_t k = i;
-      int lvl = 0;
+  if (static_cast<int>(threadIdx.x) < nv) {
+    const int64_t first = static_cast<int64_t>(blockIdx.x) * L + static_cast<int64_t>(threadIdx.x) * per;
+    double x[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = (i < per && first + i < ns) ? ssum[first + i] : 0.0;
+    if (per == 1) v = x[0];
+    else if (per == 2) v = x[0] + x[1];
+    else if (per == 4) v = (x[0] + x[1]) + (x[2] + x[3]);
+    else v = ((x[0] + x[1]) + (x[2] + x[3])) + ((x[4] + x[5]) + (x[6] + x[7]));
+  }
+  const double cta = cta_tree(v, nv, sh);
+  if (gridDim.x == 1) {
+    if (threadIdx.x == 0) *mu_out = __double2float_rn(cta / static_cast<double>(nb));
+    return;
+  }
+  if (threadIdx.x == 0) {
+    partial[blockIdx.x] = cta;
+    __threadfence();
+    is_last = (atomicAdd(ticket, 1u) == gridDim.x - 1) ? 1 : 0;
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  const int q = static_cast<int>(gridDim.x);
+  const int nv2 = q > kTreeThreads ? kTreeThreads : q;
+  const int per2 = q / nv2;                  // a power of two
+  double u = 0.0;
+  if (static_cast<int>(threadIdx.x) < nv2) {
+    // balanced sum of per2 consecutive subtree sums: a binary counter of completed subtrees
+    const volatile double* pp = partial + static_cast<int64_t>(threadIdx.x) * per2;
+    double st[32];
+    int top = 0;
+    for (int i = 0; i < per2; ++i) {
+      double x = pp[i];
+      int k = i, lvl = 0;
       while (k & 1) {
-        x = stack[lvl] + x;   // left sibling + right
+        x = st[lvl] + x;
         k >>= 1;
         ++lvl;
       }
-      stack[lvl] = x;
-      top_level = lvl;
+      st[lvl] = x;
+      top = lvl;
     }
-    v = stack[top_level];
+    u = st[top];
   }
-  s[tid] = v;
-  __syncthreads();
-  for (int len = nthreads / 2; len >= 1; len >>= 1) {
-    double x = 0.0;
-    if (tid < len) x = s[2 * tid] + s[2 * tid + 1];
-    __syncthreads();
-    if (tid < len) s[tid] = x;
-    __syncthreads();
+  const double S = cta_tree(u, nv2, sh);
+  if (threadIdx.x == 0) {
+    *mu_out = __double2float_rn(S / static_cast<double>(nb));
+    *ticket = 0u;
   }
-  if (tid == 0) *mu_out = __double2float_rn(s[0] / static_cast<double>(nblocks));
 }
 
 // Pass 2. One warp per group of 256 constants; each lane handles 8 consecutive constants.
@@ -225,6 +326,7 @@ __global__ void __launch_bounds__(256) nf4_dq_pass2(const float* __restrict__ c1
                                                     const float* __restrict__ mu_ptr,
                                                     uint8_t* __restrict__ e_out,
                                                     float* __restrict__ s2_out, int64_t ngroups) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int64_t g = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (g >= ngroups) return;
@@ -259,78 +361,130 @@ __global__ void __launch_bounds__(256) nf4_dq_pass2(const float* __restrict__ c1
   if (lane == 0) s2_out[g] = s2;
 }
 
-// Dequantize. Each thread turns 4 code bytes (8 elements) per step into 8 bf16 (16 B) or 8 fp32;
-// a warp writes 512 contiguous bytes of bf16. The 16 levels sit one per lane (16-lane segments).
+// ------------------------------------------------------------------------------------------------
+// Dequantize. A CTA owns groups (16384 elements) blockIdx.x, +gridDim.x, ...; a group's 8 KiB of codes
+// and 256 E4M3 constants come into shared memory by bulk copies kDeqStages groups ahead. Each thread
+// turns 4 code bytes (8 elements) into 16 bytes of bf16 (or 32 of fp32) per chunk; the 16 levels sit one
+// per lane (16-lane shuffle segments). A ragged last group is read straight from global memory.
+// ------------------------------------------------------------------------------------------------
 __device__ __forceinline__ float decode_e4m3(uint8_t e) {
   const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(e), __NV_E4M3);
   return __half2float(__half(h));
 }
-__device__ __forceinline__ float block_scale(const uint8_t* e4m3, const float* s2, float mu,
-                                             int64_t blk) {
-  return __fmaf_rn(decode_e4m3(e4m3[blk]), s2[blk / kGroup], mu);
+
+// The 8 values of one chunk (4 code bytes; byte b holds element 2b high, 2b+1 low). Whole warp.
+__device__ __forceinline__ void dequant8(uint32_t x, float sc, float qreg, float (&v)[8]) {
+  v[0] = __fmul_rn(lut16(qreg, x >> 4), sc);
+  v[1] = __fmul_rn(lut16(qreg, x), sc);
+  v[2] = __fmul_rn(lut16(qreg, x >> 12), sc);
+  v[3] = __fmul_rn(lut16(qreg, x >> 8), sc);
+  v[4] = __fmul_rn(lut16(qreg, x >> 20), sc);
+  v[5] = __fmul_rn(lut16(qreg, x >> 16), sc);
+  v[6] = __fmul_rn(lut16(qreg, x >> 28), sc);
+  v[7] = __fmul_rn(lut16(qreg, x >> 24), sc);
+}
+template <bool kBf16Out>
+__device__ __forceinline__ void store8(const float (&v)[8], void* __restrict__ out, int64_t chunk) {
+  if constexpr (kBf16Out) {
+    uint4 o;
+    o.x = pack_bf16x2(v[0], v[1]); o.y = pack_bf16x2(v[2], v[3]);
+    o.z = pack_bf16x2(v[4], v[5]); o.w = pack_bf16x2(v[6], v[7]);
+    __stcs(reinterpret_cast<uint4*>(out) + chunk, o);
+  } else {
+    float4* o = reinterpret_cast<float4*>(out) + 2 * chunk;
+    __stcs(o, make_float4(v[0], v[1], v[2], v[3]));
+    __stcs(o + 1, make_float4(v[4], v[5], v[6], v[7]));
+  }
 }
 
+constexpr int kDeqThreads = 256;
+constexpr int kDeqStages = 8;
+constexpr uint32_t kDeqCodeBytes = kGroupElems / 2;
+constexpr uint32_t kDeqStageBytes = kDeqCodeBytes + kGroup;
+constexpr uint32_t kDeqSmemBytes = kDeqStages * kDeqStageBytes;
+
 template <bool kBf16Out>
-__global__ void __launch_bounds__(256) nf4_dequantize_kernel(
-    const uint8_t* __restrict__ codes, const uint8_t* __restrict__ e4m3,
-    const float* __restrict__ s2, const float* __restrict__ mu_ptr, int64_t n,
-    void* __restrict__ out, CodebookArg cb) {
-  const int lane = threadIdx.x & 31;
+__global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_kernel(
+    const uint8_t* __restrict__ codes, const uint8_t* __restrict__ e4m3, const float* __restrict__ s2,
+    const float* __restrict__ mu_ptr, int64_t n, void* __restrict__ out, CodebookArg cb) {
+  extern __shared__ __align__(128) unsigned char dsm[];
+  __shared__ uint64_t bars[kDeqStages];
+  const int tid = threadIdx.x, lane = tid & 31;
   const float qreg = cb.levels[lane & 15];
   const float mu = *mu_ptr;
-  const int64_t nchunks = n / 8;                       // full 8-element chunks
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  constexpr int U = 4;
-  for (int64_t c0 = static_cast<int64_t>(blockIdx.x) * blockDim.x * U + threadIdx.x; ;
-       c0 += stride * U) {
-    // all lanes of a warp stay in the loop together (the lookups are warp-wide shuffles)
-    const int64_t warp_first = c0 - lane;
-    if (warp_first >= nchunks) break;
-    uint32_t cw[U];
-    float sc[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t c = c0 + static_cast<int64_t>(u) * blockDim.x;
-      const bool ok = c < nchunks;
-      cw[u] = ok ? __ldcs(reinterpret_cast<const uint32_t*>(codes) + c) : 0u;
-      sc[u] = ok ? block_scale(e4m3, s2, mu, (c * 8) / kBlock) : 0.0f;
+  const int64_t nfull = n / kGroupElems;
+  const int64_t ngroups = (n + kGroupElems - 1) / kGroupElems;
+  const int64_t my =
+      (static_cast<int64_t>(blockIdx.x) < ngroups) ? (ngroups - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  if (tid == 0) {
+    for (int s = 0; s < kDeqStages; ++s) mbar_init(&bars[s], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  int64_t issued = 0;   // thread 0: iterations whose copies are issued (a ragged group issues none)
+  auto issue_upto = [&](int64_t lim) {
+    for (; issued < lim && issued < my; ++issued) {
+      const int64_t g = blockIdx.x + issued * gridDim.x;
+      if (g >= nfull) continue;
+      const int s = static_cast<int>(issued % kDeqStages);
+      unsigned char* st = dsm + s * kDeqStageBytes;
+      mbar_arrive_expect_tx(&bars[s], kDeqStageBytes);
+      bulk_load(st, codes + g * kDeqCodeBytes, kDeqCodeBytes, &bars[s]);
+      bulk_load(st + kDeqCodeBytes, e4m3 + g * kGroup, kGroup, &bars[s]);
     }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t c = c0 + static_cast<int64_t>(u) * blockDim.x;
-      const uint32_t x = cw[u];
-      float v[8];
-      // byte b of x holds element 2b (high nibble) and 2b+1 (low nibble)
-      v[0] = __fmul_rn(lut16(qreg, x >> 4), sc[u]);
-      v[1] = __fmul_rn(lut16(qreg, x), sc[u]);
-      v[2] = __fmul_rn(lut16(qreg, x >> 12), sc[u]);
-      v[3] = __fmul_rn(lut16(qreg, x >> 8), sc[u]);
-      v[4] = __fmul_rn(lut16(qreg, x >> 20), sc[u]);
-      v[5] = __fmul_rn(lut16(qreg, x >> 16), sc[u]);
-      v[6] = __fmul_rn(lut16(qreg, x >> 28), sc[u]);
-      v[7] = __fmul_rn(lut16(qreg, x >> 24), sc[u]);
-      if (c < nchunks) {
-        if constexpr (kBf16Out) {
-          uint4 o;
-          o.x = pack_bf16x2(v[0], v[1]); o.y = pack_bf16x2(v[2], v[3]);
-          o.z = pack_bf16x2(v[4], v[5]); o.w = pack_bf16x2(v[6], v[7]);
-          __stcs(reinterpret_cast<uint4*>(out) + c, o);
-        } else {
-          float4* o = reinterpret_cast<float4*>(out) + 2 * c;
-          __stcs(o, make_float4(v[0], v[1], v[2], v[3]));
-          __stcs(o + 1, make_float4(v[4], v[5], v[6], v[7]));
+  };
+  if (tid == 0) issue_upto(kDeqStages);
+  int64_t i = 0;
+  int timed_out = 0;
+  for (; i < my; ++i) {
+    const int64_t g = blockIdx.x + i * gridDim.x;
+    const float sg = s2[g];
+    if (g < nfull) {
+      const int s = static_cast<int>(i % kDeqStages);
+      if (!mbar_wait(&bars[s], static_cast<uint32_t>((i / kDeqStages) & 1))) timed_out = 1;
+      const unsigned char* st = dsm + s * kDeqStageBytes;
+      const uint32_t* cw = reinterpret_cast<const uint32_t*>(st);
+      const uint8_t* ev = st + kDeqCodeBytes;
+#pragma unroll 4
+      for (int k = 0; k < kGroupElems / 8 / kDeqThreads; ++k) {
+        const int j = tid + kDeqThreads * k;           // chunk within the group; its block is j / 8
+        float v[8];
+        dequant8(cw[j], __fmaf_rn(decode_e4m3(ev[j >> 3]), sg, mu), qreg, v);
+        store8<kBf16Out>(v, out, g * (kGroupElems / 8) + j);
+      }
+    } else {
+      // ragged last group: whole 8-element chunks from global memory, then the last n % 8 elements
+      const int64_t c_end = n / 8;
+      for (int64_t cw0 = g * (kGroupElems / 8) + (tid - lane); cw0 < c_end; cw0 += kDeqThreads) {
+        const int64_t c = cw0 + lane;                  // cw0 is the warp's first chunk: warp-uniform loop
+        const bool ok = c < c_end;
+        const uint32_t x = ok ? reinterpret_cast<const uint32_t*>(codes)[c] : 0u;
+        const float sc = ok ? __fmaf_rn(decode_e4m3(e4m3[(c * 8) / kBlock]), sg, mu) : 0.0f;
+        float v[8];
+        dequant8(x, sc, qreg, v);
+        if (ok) store8<kBf16Out>(v, out, c);
+      }
+      if (tid == 0) {
+        for (int64_t e = c_end * 8; e < n; ++e) {
+          const uint8_t byte = codes[e / 2];
+          const uint32_t code = (e & 1) ? (byte & 0xFu) : (byte >> 4);
+          const float v = __fmul_rn(cb.levels[code], __fmaf_rn(decode_e4m3(e4m3[e / kBlock]), sg, mu));
+          if constexpr (kBf16Out) reinterpret_cast<__nv_bfloat16*>(out)[e] = __float2bfloat16_rn(v);
+          else reinterpret_cast<float*>(out)[e] = v;
         }
       }
     }
+    // every thread is done with the stage; the abort decision is uniform
+    if (__syncthreads_or(timed_out)) break;
+    if (tid == 0) {
+      fence_proxy_async_smem();
+      issue_upto(i + 1 + kDeqStages);
+    }
   }
-  // ragged tail (n % 8 elements): one thread, byte loads
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    for (int64_t i = nchunks * 8; i < n; ++i) {
-      const uint8_t byte = codes[i / 2];
-      const uint32_t code = (i & 1) ? (byte & 0xFu) : (byte >> 4);
-      const float v = __fmul_rn(cb.levels[code], block_scale(e4m3, s2, mu, i / kBlock));
-      if constexpr (kBf16Out) reinterpret_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(v);
-      else reinterpret_cast<float*>(out)[i] = v;
+  if (tid == 0 && i < my) {          // after a timeout: wait briefly for copies still in flight
+    for (int64_t j = i; j < issued; ++j) {
+      if (blockIdx.x + j * gridDim.x < nfull)
+        mbar_wait_short(&bars[j % kDeqStages], static_cast<uint32_t>((j / kDeqStages) & 1));
     }
   }
 }

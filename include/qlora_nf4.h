@@ -108,7 +108,8 @@ int qlora_nf4_quantize_workspace(int64_t n, size_t* bytes);
  *   3. per group of 256 blocks: d = c1 - mu (fp32), s2 = max|d| / 448 (fp32), e = E4M3 round-to-nearest-
  *      even, saturating, of d / s2 (e = 0 when s2 = 0).
  * Any numel >= 1 is accepted; the last block and group may be partial. `workspace` (device, >=
- * qlora_nf4_quantize_workspace bytes) holds the fp32 c1 and per-group partial sums between passes.
+ * qlora_nf4_quantize_workspace bytes) holds the fp32 c1, fp64 partial sums of the mean's tree and an
+ * arrival counter between passes; its contents need no initialisation and are not kept between calls.
  * A non-finite input sets QLORA_STATUS_NONFINITE; the outputs of that call are then unspecified.
  * Results are deterministic and bit-identical run to run.
  */
@@ -124,7 +125,7 @@ int qlora_nf4_quantize(const void* w, int w_dtype, int64_t rows, int64_t cols,
  * framework's caching allocator, where a cudaMalloc behind the framework's back can synchronize the
  * device and fragment memory the framework manages; plugin or callback interfaces that hand over only
  * the input and output buffers; and loops that forbid allocation after start-up. The caller still
- * allocates `out` (qlora_nf4_storage_bytes); the intermediate per-block constants and per-group sums live
+ * allocates `out` (qlora_nf4_storage_bytes); the intermediate per-block constants and partial sums live
  * in one fixed scratch array inside the library, QLORA_NOALLOC_SCRATCH_BYTES (about 4 MiB) of device
  * memory that every GPU which loads the library holds until the process exits.
  *   - rows * cols must not exceed QLORA_NOALLOC_MAX_NUMEL (2^26); larger inputs return
@@ -138,7 +139,7 @@ int qlora_nf4_quantize(const void* w, int w_dtype, int64_t rows, int64_t cols,
  * Other arguments, checks, status reporting and results are those of qlora_nf4_quantize.
  */
 #define QLORA_NOALLOC_MAX_NUMEL (((int64_t)1) << 26)
-#define QLORA_NOALLOC_SCRATCH_BYTES ((size_t)4 * 1024 * 1024 + (size_t)8 * 4096)
+#define QLORA_NOALLOC_SCRATCH_BYTES ((size_t)4 * 1024 * 1024 + (size_t)128 * 1024 + (size_t)512)
 int qlora_nf4_quantize_noalloc(const void* w, int w_dtype, int64_t rows, int64_t cols,
                                const qlora_nf4_tensor* out, qlora_stream_t stream);
 

@@ -138,3 +138,59 @@ def test_deterministic(lib):
     b = lib.quantize(torch.from_numpy(x).cuda())
     for f in ("codes", "absmax_e4m3", "scale2", "offset"):
         assert torch.equal(getattr(a, f), getattr(b, f))
+
+
+def _rd_f32(p):
+    """fp32 rounding toward -inf of the exactly representable fp64 values p."""
+    f = p.astype(np.float32)
+    down = f.astype(np.float64) > p
+    f[down] = np.nextafter(f[down], np.float32(-np.inf))
+    return f
+
+
+ABSMAX = [1.0, 0.02, 3.7e-3, 0.5, 448.0, 2.0 ** -100, 2.0 ** -126, 1e-39, 3e38]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_codes_over_every_bf16_value(lib, dtype):
+    """For absmax values a from subnormal to near the fp32 maximum, every finite bf16 value w with
+    |w| <= a, in blocks led by +a or -a (so a is the block absmax): codes, constants and the dequantized
+    values equal the oracle's exact threshold rule. With fp32 input, also the 7 fp32 values around each
+    decision point RD(T_j a) for every threshold j. Covers every bucket of the table-assisted code search,
+    the scaled path for absmax below 2^-120, and reciprocals that are subnormal (a near 3e38)."""
+    _, T = O.nf4_codebook()
+    allv = (np.arange(65536, dtype=np.uint32) << 16).view(np.float32)
+    allv = allv[np.isfinite(allv)]
+    blocks = []
+    for a0 in ABSMAX:
+        a = np.float32(a0)
+        if dtype == "bf16":
+            a = synth.bf16_values(synth.to_bf16(np.array([a], np.float32)))[0]
+        vals = allv[np.abs(allv) <= a]
+        if dtype == "f32":
+            P = _rd_f32(T.astype(np.float64) * np.float64(a))
+            near = [P]
+            up, dn = P.copy(), P.copy()
+            for _ in range(3):
+                up = np.nextafter(up, np.float32(np.inf))
+                dn = np.nextafter(dn, np.float32(-np.inf))
+                near += [up.copy(), dn.copy()]
+            near = np.concatenate(near)
+            vals = np.concatenate([vals, near[np.abs(near) <= a]])
+        for sign in (1.0, -1.0):
+            pad = (-len(vals)) % 63
+            body = np.concatenate([vals, np.zeros(pad, np.float32)]).reshape(-1, 63)
+            lead = np.full((body.shape[0], 1), np.float32(sign) * a, np.float32)
+            blocks.append(np.concatenate([lead, body], axis=1).reshape(-1))
+    x = np.concatenate(blocks).astype(np.float32)
+    if dtype == "f32":
+        q, st = run_quantize(lib, x)
+        ref = O.quantize(x)
+    else:
+        xb = synth.to_bf16(x)
+        assert np.array_equal(synth.bf16_values(xb), x)          # every value is bf16-exact
+        q, st = run_quantize(lib, w_t=xb.cuda())
+        ref = O.quantize(synth.bf16_bits(xb))
+    assert st == 0
+    assert_same_as_oracle(q, ref)
+    assert_dequant_same(lib, q, ref, x.shape)
