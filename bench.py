@@ -349,6 +349,8 @@ def run_gpu(args):
     for _ in range(args.steps):
         run_step(q, wl)
     ev1.record(stream)
+    while not ev1.query():          # poll with sleeps so the sampler thread gets the interpreter
+        time.sleep(0.0005)
     torch.cuda.synchronize()
     barrier(device)
     launches = q.kernel_launches() - n0
