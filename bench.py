@@ -24,6 +24,7 @@ import argparse
 import datetime
 import hashlib
 import json
+import math
 import os
 import statistics
 import sys
@@ -443,6 +444,128 @@ def emit(args, world, ms_max, value, e2e, launches, prof, clk, status, wl):
     print(json.dumps(line), flush=True)
 
 
+# ---- secondary workloads: decode-shaped forward and the codec sweep ------------------------------
+# (python bench.py --workload decode | codec_sweep; one JSON line each, with every case listed)
+
+DECODE_TOKENS = (1, 4, 16)
+DECODE_WORKLOAD = ("LLaMA-65B-shaped frozen NF4 linears (N x K = 8192x8192, 22016x8192, 8192x22016), "
+                   "forward only at T = 1, 4, 16 tokens, r = 64, alpha = 16")
+SWEEP_SIZES = tuple(2 ** e for e in (20, 22, 24, 26, 28, 30))
+
+
+def gemv_bytes(T, N, K, r):
+    """Algorithmic HBM bytes of one decode-shaped forward: the stored NF4 weight, A and B, X in, Y out."""
+    return (0.5 + 1 / 64 + 4 / 16384) * N * K + 2 * r * (N + K) + 2 * T * (N + K)
+
+
+def time_calls(fn, flush, reps, warmup=3):
+    """Median device time (ms) of fn() over reps calls, the L2 flushed by a 512 MB write before each
+    (outside the timed pair of events, on the same stream)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    stream = torch.cuda.current_stream()
+    times = []
+    for i in range(reps):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    return statistics.median(times)
+
+
+def run_decode(args):
+    import torch
+    import synth
+    import bit_nf4_quantized_14_b200 as q
+    peaks, kind = load_peaks()
+    device = torch.device("cuda", 0)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    cases = []
+    for i, (N, K) in enumerate(synth.LLAMA65B_SHAPES):
+        W = torch.from_numpy(synth.weight_f32(N, K, seed=40 + i, tensor_id=1)).to(device)
+        nf4 = q.quantize(W)
+        del W
+        A = synth.to_bf16(synth.normal_f32((RANK_R, K), 0.01, 40 + i, 3)).to(device)
+        B = synth.to_bf16(synth.normal_f32((N, RANK_R), 0.01, 40 + i, 4)).to(device)
+        X16 = synth.to_bf16(synth.normal_f32((max(DECODE_TOKENS), K), 1.0, 40 + i, 2)).to(device)
+        for T in DECODE_TOKENS:
+            X = X16[:T].contiguous()
+            Y = torch.empty(T, N, dtype=torch.bfloat16, device=device)
+            U = torch.empty(T, RANK_R, dtype=torch.bfloat16, device=device)
+            ws = torch.empty(q.linear_workspace_bytes(T, N, K, RANK_R), dtype=torch.uint8, device=device)
+            fn = lambda: q.linear_fwd(X, nf4, A, B, ALPHA, out=Y, U_out=U, workspace=ws)
+            n0 = q.kernel_launches()
+            fn()
+            launches = q.kernel_launches() - n0
+            ms = time_calls(fn, flush, args.steps, args.warmup)
+            gbs = gemv_bytes(T, N, K, RANK_R) / (ms / 1e3) / 1e9
+            cases.append({"N": N, "K": K, "T": T, "us": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
+                          "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes": int(gemv_bytes(T, N, K, RANK_R)),
+                          "launches_per_call": launches})
+    status = q.get_status()
+    gm = math.exp(sum(math.log(c["GB/s"]) for c in cases) / len(cases))
+    print(json.dumps({"metric": "QLoRA decode-shaped linear forward, HBM GB/s (geomean over cases)",
+                      "value": round(gm, 1), "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+                      "warmup": args.warmup, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+                      "config": {"workload": DECODE_WORKLOAD, "r": RANK_R, "alpha": ALPHA,
+                                 "l2": "flushed (512 MB write) before every timed call"},
+                      "roofline": {"bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                                   "peak_source": f"{kind} (HBM copy)", "achieved": round(gm, 1),
+                                   "frac": round(gm / peaks["hbm_gbs"], 4)},
+                      "cases": cases, "device_status": status}), flush=True)
+    return 0
+
+
+def run_codec_sweep(args):
+    import torch
+    import synth
+    import bit_nf4_quantized_14_b200 as q
+    peaks, kind = load_peaks()
+    device = torch.device("cuda", 0)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    chunk = 1 << 28          # the largest sizes are concatenations of independent 2^28-element sweep tensors
+    nmax = max(SWEEP_SIZES)
+    x = torch.empty(nmax, dtype=torch.float32, device=device)
+    for c in range(0, nmax, chunk):
+        m = min(chunk, nmax - c)
+        x[c:c + m] = torch.from_numpy(synth.sweep_f32(m, seed=50, tensor_id=c // chunk)).to(device)
+    xb = x.to(torch.bfloat16)
+    cases = []
+    for n in SWEEP_SIZES:
+        out = q.NF4Weight.empty(1, n, device)
+        ws = torch.empty(q.quantize_workspace_bytes(n), dtype=torch.uint8, device=device)
+        deq = torch.empty(1, n, dtype=torch.bfloat16, device=device)
+        row = {"n": n}
+        for name, src, bpe in (("quantize_fp32", x[:n].view(1, n), 4 + DEQ_B_PER_ELEM - 2),
+                               ("quantize_bf16", xb[:n].view(1, n), 2 + DEQ_B_PER_ELEM - 2)):
+            ms = time_calls(lambda: q.quantize(src, out=out, workspace=ws), flush, args.steps, args.warmup)
+            row[name] = {"us": round(ms * 1e3, 2), "GB/s": round(n * bpe / (ms / 1e3) / 1e9, 1),
+                         "frac": round(n * bpe / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
+        ms = time_calls(lambda: q.dequantize(out, torch.bfloat16, out=deq), flush, args.steps, args.warmup)
+        row["dequantize_bf16"] = {"us": round(ms * 1e3, 2), "GB/s": round(n * DEQ_B_PER_ELEM / (ms / 1e3) / 1e9, 1),
+                                  "frac": round(n * DEQ_B_PER_ELEM / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
+        cases.append(row)
+        del out, ws, deq
+    status = q.get_status()
+    top = cases[-1]
+    print(json.dumps({"metric": "NF4 quantize / dequantize HBM GB/s over the size sweep (value: fp32 quantize "
+                                "at the largest size)",
+                      "value": top["quantize_fp32"]["GB/s"], "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+                      "warmup": args.warmup, "higher_is_better": True, "dtype": "f32/bf16 in, u8 + e4m3 out",
+                      "data": "synthetic",
+                      "config": {"workload": "sweep tensors: rows of 4096, sigma_row ~ U(0.005, 0.05), 0.1 % x10 "
+                                             "outliers; sizes 2^20..2^30 (2^30 = four 2^28 sweeps)",
+                                 "l2": "flushed (512 MB write) before every timed call"},
+                      "roofline": {"bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                                   "peak_source": f"{kind} (HBM copy)"},
+                      "cases": cases, "device_status": status}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -451,6 +574,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) measurement")
+    ap.add_argument("--workload", choices=["llama7b_step", "decode", "codec_sweep"], default="llama7b_step",
+                    help="llama7b_step (the headline line), or the decode / codec-sweep measurement lines")
     ap.add_argument("--shapes", default="all",
                     help="comma-separated NxK subset of the workload shapes (profiling runs), e.g. 4096x4096")
     args = ap.parse_args(argv)
@@ -461,6 +586,10 @@ def main(argv=None):
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "decode":
+        return run_decode(args)
+    if args.workload == "codec_sweep":
+        return run_codec_sweep(args)
     return run_gpu(args)
 
 

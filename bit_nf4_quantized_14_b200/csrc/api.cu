@@ -13,6 +13,7 @@
 #include "codec.cuh"
 #include "gemm_nf4w.cuh"
 #include "gemm_sm100.cuh"
+#include "gemv_nf4.cuh"
 
 namespace qnf4 {
 void build_nf4_codebook(float levels[16], float thresholds[15]);   // codebook.cpp
@@ -318,9 +319,47 @@ int check_nf4(const qlora_nf4_tensor* q) {
 }
 
 struct LinearWs { size_t sU, sV, scales, part, total; };
+// ---- small-token path (T <= kGvMaxTokens): the stream-K GEMV kernels ---------------------------
+constexpr int kGvMaxCtas = 256;          // grid cap of the GEMV launches (>= the SM count of any B200)
+constexpr int kGvDenseCtas = 16;         // grid cap of the adapter projection (sU)
+inline int gv_nt(int64_t T) { return T <= 8 ? 1 : T <= 16 ? 2 : T <= 32 ? 4 : 8; }
+struct GvShape { int spt, tiles; int64_t total; };
+inline GvShape gv_shape(int64_t rows, int64_t K, bool dense) {
+  GvShape g;
+  g.spt = static_cast<int>(dense ? K / 64 : cdiv(K, 256));
+  g.tiles = static_cast<int>(cdiv(rows, kGvRows));
+  g.total = static_cast<int64_t>(g.spt) * g.tiles;
+  return g;
+}
+inline int gv_maxseg(const GvShape& g, int G) {
+  return static_cast<int>(cdiv(cdiv(g.total, G), g.spt)) + 1;
+}
+// Partial slots a launch of up to `cap` CTAs can need (the largest G * maxseg over G <= cap).
+inline int64_t gv_slots(const GvShape& g, int cap) {
+  int64_t best = 0;
+  for (int G = 1; G <= std::min<int64_t>(cap, g.total); ++G) best = std::max<int64_t>(best, int64_t(G) * gv_maxseg(g, G));
+  return best;
+}
+// Layout inside the linear workspace's fp32 region (offsets in bytes): NF4 partials, adapter partials,
+// then the two ticket arrays (one counter per tile and consumer warp).
+struct GemvWs { size_t part_w, part_u, ticket_w, ticket_u, ticket_bytes, total; };
+GemvWs gemv_ws(int64_t T, int64_t N, int64_t K, int r) {
+  const int64_t slot = int64_t(kGvWarps) * 32 * gv_nt(T) * 4 * 4;      // bytes of one partial tile
+  const GvShape gw = gv_shape(N, K, false), gu = gv_shape(r, K, true);
+  GemvWs w;
+  w.part_w = 0;
+  w.part_u = align256(static_cast<size_t>(gv_slots(gw, kGvMaxCtas) * slot));
+  w.ticket_w = w.part_u + align256(static_cast<size_t>(gv_slots(gu, kGvDenseCtas) * slot));
+  w.ticket_u = w.ticket_w + align256(static_cast<size_t>(gw.tiles) * kGvWarps * 4);
+  w.total = w.ticket_u + align256(static_cast<size_t>(gu.tiles) * kGvWarps * 4);
+  w.ticket_bytes = w.total - w.ticket_w;
+  return w;
+}
+
 LinearWs linear_ws(int64_t T, int64_t N, int64_t K, int r) {
   const int bn = static_cast<int>(cdiv(r, 64) * 64);
   int64_t part = 0;
+  if (T <= kGvMaxTokens) part = static_cast<int64_t>(gemv_ws(T, N, K, r).total / 4);
   part = std::max(part, skinny_part_elems(T, K, bn));   // U
   part = std::max(part, skinny_part_elems(T, N, bn));   // V
   part = std::max(part, skinny_part_elems(K, T, bn));   // dA
@@ -348,6 +387,95 @@ int check_linear(const void* X, int64_t T, const qlora_nf4_tensor* W, const void
 }
 
 // sU = s * X A^T (T x r, bf16) via the split adapter GEMM and its reduction.
+template <int NT, bool kDense>
+int launch_gemv_nt(const CUtensorMap& ta, const CUtensorMap& tx, const GvParams& p, int grid, bool pdl,
+                   cudaStream_t st) {
+  using C = GvCfg<NT, kDense>;
+  auto kern = nf4_gemv_kernel<NT, kDense>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGvThreads);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tx, p, codebook()) != cudaSuccess) return QLORA_ERR_CUDA;
+  return launched();
+}
+template <bool kDense>
+int launch_gemv(int nt, const CUtensorMap& ta, const CUtensorMap& tx, const GvParams& p, int grid, bool pdl,
+                cudaStream_t st) {
+  switch (nt) {
+    case 1: return launch_gemv_nt<1, kDense>(ta, tx, p, grid, pdl, st);
+    case 2: return launch_gemv_nt<2, kDense>(ta, tx, p, grid, pdl, st);
+    case 4: return launch_gemv_nt<4, kDense>(ta, tx, p, grid, pdl, st);
+    default: return launch_gemv_nt<8, kDense>(ta, tx, p, grid, pdl, st);
+  }
+}
+GvParams gv_params(int64_t T, int64_t rows, int64_t K, const GvShape& g, int G) {
+  GvParams p = {};
+  p.T = static_cast<int>(T);
+  p.rows = static_cast<int>(rows);
+  p.K = static_cast<int>(K);
+  p.spt = g.spt;
+  p.tiles = g.tiles;
+  p.total = g.total;
+  p.maxseg = gv_maxseg(g, G);
+  return p;
+}
+
+// sU = s * X A^T for T <= kGvMaxTokens by the dense GEMV; clears both GEMV ticket arrays first.
+int gemv_sU(const void* X, int64_t T, int64_t K, const void* A, int r, float s, void* sU, char* gws,
+            const GemvWs& L, cudaStream_t st) {
+  if (cudaMemsetAsync(gws + L.ticket_w, 0, L.ticket_bytes, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  const int nt = gv_nt(T);
+  CUtensorMap ta, tx;
+  if (!make_tmap_t(&ta, A, TmType::kBf16, K, r, K, 64, kGvRows, true) ||
+      !make_tmap_t(&tx, X, TmType::kBf16, K, T, K, 64, 8 * nt, true))
+    return QLORA_ERR_CUDA;
+  const GvShape g = gv_shape(r, K, true);
+  const int G = static_cast<int>(std::min<int64_t>(g.total, kGvDenseCtas));
+  GvParams p = gv_params(T, r, K, g, G);
+  p.out_scale = s;
+  p.out = static_cast<__nv_bfloat16*>(sU);
+  p.ldo = r;
+  p.part = reinterpret_cast<float*>(gws + L.part_u);
+  p.ticket = reinterpret_cast<unsigned*>(gws + L.ticket_u);
+  return launch_gemv<true>(nt, ta, tx, p, G, false, st);
+}
+
+// Y = X W_hat^T + sU B^T for T <= kGvMaxTokens (after gemv_sU on the same stream).
+int gemv_fwd(const void* X, int64_t T, const qlora_nf4_tensor* W, const void* B, int r, const void* sU, void* Y,
+             char* gws, const GemvWs& L, int sms, cudaStream_t st) {
+  const int64_t N = W->rows, K = W->cols;
+  const int nt = gv_nt(T);
+  CUtensorMap ta, tx;
+  if (!make_tmap_t(&ta, W->codes, TmType::kU8, K / 2, N, K / 2, 128, kGvRows, true) ||
+      !make_tmap_t(&tx, X, TmType::kBf16, K, T, K, 64, 8 * nt, true))
+    return QLORA_ERR_CUDA;
+  const GvShape g = gv_shape(N, K, false);
+  const int G = static_cast<int>(std::min<int64_t>(std::min<int64_t>(g.total, sms), kGvMaxCtas));
+  GvParams p = gv_params(T, N, K, g, G);
+  p.kbw = static_cast<int>(K / 64);
+  p.e4m3 = W->absmax_e4m3;
+  p.s2 = W->scale2;
+  p.mu = W->offset;
+  p.sU = static_cast<const __nv_bfloat16*>(sU);
+  p.Bw = static_cast<const __nv_bfloat16*>(B);
+  p.r = r;
+  p.out_scale = 1.0f;
+  p.out = static_cast<__nv_bfloat16*>(Y);
+  p.ldo = N;
+  p.part = reinterpret_cast<float*>(gws + L.part_w);
+  p.ticket = reinterpret_cast<unsigned*>(gws + L.ticket_w);
+  return launch_gemv<false>(nt, ta, tx, p, G, true, st);
+}
+
 int compute_sU(const void* X, int64_t T, int64_t K, const void* A, int r, float s, void* sU, float* part,
                cudaStream_t st) {
   const int bn = static_cast<int>(cdiv(r, 64) * 64);
@@ -533,6 +661,17 @@ int qlora_linear_fwd(const void* X, int64_t T, const qlora_nf4_tensor* W, const 
   char* ws = static_cast<char*>(workspace);
   void* sU = U_out ? U_out : ws + L.sU;
   float* part = reinterpret_cast<float*>(ws + L.part);
+  if (T <= kGvMaxTokens) {                      // decode-sized: the stream-K GEMV kernels
+    int sms = 0;
+    if (int e = check_device(&sms)) return e;
+    const GemvWs G = gemv_ws(T, N, K, r);
+    {
+      ProfScope prof(QLORA_PROF_LORA, st);
+      if (int e = gemv_sU(X, T, K, A, r, s, sU, ws + L.part, G, st)) return e;
+    }
+    ProfScope prof(QLORA_PROF_FWD_GEMM, st);
+    return gemv_fwd(X, T, W, B, r, sU, Y, ws + L.part, G, sms, st);
+  }
   {
     ProfScope prof(QLORA_PROF_LORA, st);
     if (int e = compute_sU(X, T, K, A, r, s, sU, part, st)) return e;
@@ -560,8 +699,12 @@ int qlora_linear_bwd(const void* dY, const void* X, int64_t T, const qlora_nf4_t
   const void* sU = U;
   {
     ProfScope prof(QLORA_PROF_LORA, st);
-    if (!sU) {
-      if (int e = compute_sU(X, T, K, A, r, s, ws + L.sU, part, st)) return e;
+    if (!sU) {                                  // the forward's own projection, so U is identical
+      if (T <= kGvMaxTokens) {
+        if (int e = gemv_sU(X, T, K, A, r, s, ws + L.sU, ws + L.part, gemv_ws(T, N, K, r), st)) return e;
+      } else if (int e = compute_sU(X, T, K, A, r, s, ws + L.sU, part, st)) {
+        return e;
+      }
       sU = ws + L.sU;
     }
     // sV = s * dY B  (T x r): contraction over the N output features; B is N x r, i.e. MN-major.

@@ -131,3 +131,60 @@ def test_persistent_tiles_full_compare(lib, N, K):
     shared-memory ring and both tensor-memory accumulators. Every output is compared."""
     case = synth.linear_case(T=4096, N=N, K=K, r=64, alpha=16.0, seed=6)
     run_and_check(lib, case)
+
+
+# ---- small token counts (decode shapes): the stream-K GEMV path serves T <= 64 --------------------
+
+@pytest.mark.parametrize("T", [1, 2, 4, 7, 8, 9, 16, 17, 32, 33, 64])
+@pytest.mark.parametrize("N,K,r", [(520, 704, 24), (1000, 320, 64)])
+def test_small_token_forward(lib, T, N, K, r):
+    """T <= 64 runs the GEMV kernels: tails in rows (240-row tiles), in the contraction (256-wide stages),
+    in tokens (8-wide MMA tiles) and in r (16-deep MMA steps). Y and U against the oracle; the backward
+    (GEMM path) against the oracle as well, with U from this forward and recomputed."""
+    case = synth.linear_case(T=T, N=N, K=K, r=r, alpha=16.0, seed=11 + T)
+    errs, (Y, U, dX, dA, dB), q, d = run_and_check(lib, case)
+    dX2, dA2, dB2 = lib.linear_bwd(d["dY"], d["X"], q, d["A"], d["B"], 16.0, U=None)
+    assert torch.equal(dA, dA2) and torch.equal(dB, dB2)
+
+
+@pytest.mark.parametrize("T", [1, 16])
+def test_small_token_adapter_only_and_base_only(lib, T):
+    case = synth.linear_case(T=T, N=496, K=448, r=16, alpha=16.0, seed=21, zero_w=True)
+    errs, (Y, U, dX, dA, dB), *_ = run_and_check(lib, case)
+    assert float(Y.float().abs().max()) > 0
+    case = synth.linear_case(T=T, N=496, K=448, r=16, alpha=16.0, seed=22, zero_b=True)
+    q, Wt, d, h = setup(lib, case)
+    Y, U = lib.linear_fwd(d["X"], q, d["A"], d["B"], 16.0)
+    Yr = h["X"].astype(np.float64) @ Wt.T.astype(np.float64)
+    assert rel(Y.float().cpu(), Yr) <= TOL
+
+
+def test_small_token_deterministic(lib):
+    case = synth.linear_case(T=5, N=2048, K=4096, r=64, alpha=16.0, seed=23)
+    q, Wt, d, h = setup(lib, case)
+    outs = [lib.linear_fwd(d["X"], q, d["A"], d["B"], 16.0) for _ in range(3)]
+    for o in outs[1:]:
+        assert torch.equal(outs[0][0], o[0]) and torch.equal(outs[0][1], o[1])
+
+
+@pytest.mark.parametrize("T", [64, 65])
+def test_gemv_and_gemm_paths_at_the_boundary(lib, T):
+    """T = 64 is the last GEMV size, T = 65 the first fused-GEMM size: both meet the oracle's tolerance on
+    the same layer, so the two paths agree with each other to twice it."""
+    case = synth.linear_case(T=T, N=1024, K=1024, r=64, alpha=16.0, seed=24)
+    run_and_check(lib, case)
+
+
+@pytest.mark.parametrize("N,K,Ts", [(8192, 8192, (1, 4, 16)), (4096, 11008, (16,))])
+def test_decode_shapes(lib, N, K, Ts):
+    """The decode-shaped layers (65B-sized 8192 x 8192; the wide contraction of a down projection) at the
+    decode token counts: every output of Y and U against the oracle (fp64 GEMM over the exact W_hat)."""
+    case = synth.linear_case(T=max(Ts), N=N, K=K, r=64, alpha=16.0, seed=25)
+    q, Wt, d, h = setup(lib, case)
+    for T in Ts:
+        X = d["X"][:T].contiguous()
+        Y, U = lib.linear_fwd(X, q, d["A"], d["B"], 16.0)
+        assert lib.get_status() == 0
+        Yr, Ur = O.linear_fwd(h["X"][:T], Wt, h["A"], h["B"], 16.0)
+        assert rel(Y.float().cpu(), Yr) <= TOL, T
+        assert rel(U.float().cpu(), (16.0 / 64) * Ur) <= TOL, T
