@@ -320,13 +320,13 @@ int check_nf4(const qlora_nf4_tensor* q) {
 
 struct LinearWs { size_t sU, sV, scales, part, total; };
 // ---- small-token path (T <= kGvMaxTokens): the stream-K GEMV kernels ---------------------------
-constexpr int kGvMaxCtas = 256;          // grid cap of the GEMV launches (>= the SM count of any B200)
-constexpr int kGvDenseCtas = 16;         // grid cap of the adapter projection (sU)
+constexpr int kGvMaxCtas = 256;          // grid cap of the NF4 GEMV (>= the SM count of any B200)
+constexpr int kGuMaxSlices = 32;         // contraction slices of the adapter projection
 inline int gv_nt(int64_t T) { return T <= 8 ? 1 : T <= 16 ? 2 : T <= 32 ? 4 : 8; }
 struct GvShape { int spt, tiles; int64_t total; };
-inline GvShape gv_shape(int64_t rows, int64_t K, bool dense) {
+inline GvShape gv_shape(int64_t rows, int64_t K) {
   GvShape g;
-  g.spt = static_cast<int>(dense ? K / 64 : cdiv(K, 256));
+  g.spt = static_cast<int>(cdiv(K, kGvStageK));
   g.tiles = static_cast<int>(cdiv(rows, kGvRows));
   g.total = static_cast<int64_t>(g.spt) * g.tiles;
   return g;
@@ -340,18 +340,29 @@ inline int64_t gv_slots(const GvShape& g, int cap) {
   for (int G = 1; G <= std::min<int64_t>(cap, g.total); ++G) best = std::max<int64_t>(best, int64_t(G) * gv_maxseg(g, G));
   return best;
 }
+struct GuShape { int groups, kslices, kb_per_slice; };
+inline GuShape gu_shape(int64_t K, int r) {
+  const int nkb = static_cast<int>(K / 64);
+  GuShape u;
+  u.groups = static_cast<int>(cdiv(r, 16));
+  u.kb_per_slice = static_cast<int>(cdiv(nkb, std::min(nkb, kGuMaxSlices)));
+  u.kslices = static_cast<int>(cdiv(nkb, u.kb_per_slice));
+  return u;
+}
 // Layout inside the linear workspace's fp32 region (offsets in bytes): NF4 partials, adapter partials,
-// then the two ticket arrays (one counter per tile and consumer warp).
+// then the two ticket arrays (NF4: one per tile and consumer warp; adapter: one per 16 rows).
 struct GemvWs { size_t part_w, part_u, ticket_w, ticket_u, ticket_bytes, total; };
 GemvWs gemv_ws(int64_t T, int64_t N, int64_t K, int r) {
-  const int64_t slot = int64_t(kGvWarps) * 32 * gv_nt(T) * 4 * 4;      // bytes of one partial tile
-  const GvShape gw = gv_shape(N, K, false), gu = gv_shape(r, K, true);
+  const int nt = gv_nt(T);
+  const int64_t slot = int64_t(kGvWarps) * 32 * nt * 4 * 4;      // bytes of one partial tile
+  const GvShape gw = gv_shape(N, K);
+  const GuShape gu = gu_shape(K, r);
   GemvWs w;
   w.part_w = 0;
   w.part_u = align256(static_cast<size_t>(gv_slots(gw, kGvMaxCtas) * slot));
-  w.ticket_w = w.part_u + align256(static_cast<size_t>(gv_slots(gu, kGvDenseCtas) * slot));
+  w.ticket_w = w.part_u + align256(static_cast<size_t>(gu.groups) * gu.kslices * 32 * nt * 4 * 4);
   w.ticket_u = w.ticket_w + align256(static_cast<size_t>(gw.tiles) * kGvWarps * 4);
-  w.total = w.ticket_u + align256(static_cast<size_t>(gu.tiles) * kGvWarps * 4);
+  w.total = w.ticket_u + align256(static_cast<size_t>(gu.groups) * 4);
   w.ticket_bytes = w.total - w.ticket_w;
   return w;
 }
@@ -387,11 +398,10 @@ int check_linear(const void* X, int64_t T, const qlora_nf4_tensor* W, const void
 }
 
 // sU = s * X A^T (T x r, bf16) via the split adapter GEMM and its reduction.
-template <int NT, bool kDense>
-int launch_gemv_nt(const CUtensorMap& ta, const CUtensorMap& tx, const GvParams& p, int grid, bool pdl,
-                   cudaStream_t st) {
-  using C = GvCfg<NT, kDense>;
-  auto kern = nf4_gemv_kernel<NT, kDense>;
+template <int NT>
+int launch_gemv_nt(const CUtensorMap& ta, const CUtensorMap& tx, const GvParams& p, int grid, cudaStream_t st) {
+  using C = GvCfg<NT>;
+  auto kern = nf4_gemv_kernel<NT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return QLORA_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
@@ -399,68 +409,61 @@ int launch_gemv_nt(const CUtensorMap& ta, const CUtensorMap& tx, const GvParams&
   cfg.blockDim = dim3(kGvThreads);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[1];               // may start while the adapter projection runs
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, ta, tx, p, codebook()) != cudaSuccess) return QLORA_ERR_CUDA;
   return launched();
 }
-template <bool kDense>
-int launch_gemv(int nt, const CUtensorMap& ta, const CUtensorMap& tx, const GvParams& p, int grid, bool pdl,
-                cudaStream_t st) {
-  switch (nt) {
-    case 1: return launch_gemv_nt<1, kDense>(ta, tx, p, grid, pdl, st);
-    case 2: return launch_gemv_nt<2, kDense>(ta, tx, p, grid, pdl, st);
-    case 4: return launch_gemv_nt<4, kDense>(ta, tx, p, grid, pdl, st);
-    default: return launch_gemv_nt<8, kDense>(ta, tx, p, grid, pdl, st);
-  }
-}
-GvParams gv_params(int64_t T, int64_t rows, int64_t K, const GvShape& g, int G) {
-  GvParams p = {};
-  p.T = static_cast<int>(T);
-  p.rows = static_cast<int>(rows);
-  p.K = static_cast<int>(K);
-  p.spt = g.spt;
-  p.tiles = g.tiles;
-  p.total = g.total;
-  p.maxseg = gv_maxseg(g, G);
-  return p;
-}
 
-// sU = s * X A^T for T <= kGvMaxTokens by the dense GEMV; clears both GEMV ticket arrays first.
+// sU = s * X A^T for T <= kGvMaxTokens; clears both ticket arrays of the small-token path first.
 int gemv_sU(const void* X, int64_t T, int64_t K, const void* A, int r, float s, void* sU, char* gws,
             const GemvWs& L, cudaStream_t st) {
   if (cudaMemsetAsync(gws + L.ticket_w, 0, L.ticket_bytes, st) != cudaSuccess) return QLORA_ERR_CUDA;
-  const int nt = gv_nt(T);
-  CUtensorMap ta, tx;
-  if (!make_tmap_t(&ta, A, TmType::kBf16, K, r, K, 64, kGvRows, true) ||
-      !make_tmap_t(&tx, X, TmType::kBf16, K, T, K, 64, 8 * nt, true))
-    return QLORA_ERR_CUDA;
-  const GvShape g = gv_shape(r, K, true);
-  const int G = static_cast<int>(std::min<int64_t>(g.total, kGvDenseCtas));
-  GvParams p = gv_params(T, r, K, g, G);
-  p.out_scale = s;
-  p.out = static_cast<__nv_bfloat16*>(sU);
-  p.ldo = r;
+  const GuShape u = gu_shape(K, r);
+  GuParams p = {};
+  p.T = static_cast<int>(T);
+  p.r = r;
+  p.K = static_cast<int>(K);
+  p.kslices = u.kslices;
+  p.kb_per_slice = u.kb_per_slice;
+  p.X = static_cast<const __nv_bfloat16*>(X);
+  p.A = static_cast<const __nv_bfloat16*>(A);
+  p.s = s;
+  p.sU = static_cast<__nv_bfloat16*>(sU);
   p.part = reinterpret_cast<float*>(gws + L.part_u);
   p.ticket = reinterpret_cast<unsigned*>(gws + L.ticket_u);
-  return launch_gemv<true>(nt, ta, tx, p, G, false, st);
+  const dim3 grid(u.groups, u.kslices);
+  switch (gv_nt(T)) {
+    case 1: lora_u_kernel<1><<<grid, 32, 0, st>>>(p); break;
+    case 2: lora_u_kernel<2><<<grid, 32, 0, st>>>(p); break;
+    case 4: lora_u_kernel<4><<<grid, 32, 0, st>>>(p); break;
+    default: lora_u_kernel<8><<<grid, 32, 0, st>>>(p); break;
+  }
+  return launched();
 }
 
-// Y = X W_hat^T + sU B^T for T <= kGvMaxTokens (after gemv_sU on the same stream).
+// Y = X W_hat^T + sU B^T for T <= kGvMaxTokens (right after gemv_sU on the same stream).
 int gemv_fwd(const void* X, int64_t T, const qlora_nf4_tensor* W, const void* B, int r, const void* sU, void* Y,
              char* gws, const GemvWs& L, int sms, cudaStream_t st) {
   const int64_t N = W->rows, K = W->cols;
   const int nt = gv_nt(T);
   CUtensorMap ta, tx;
-  if (!make_tmap_t(&ta, W->codes, TmType::kU8, K / 2, N, K / 2, 128, kGvRows, true) ||
+  if (!make_tmap_t(&ta, W->codes, TmType::kU8, K / 2, N, K / 2, kGvRowBytes, kGvRows, true) ||
       !make_tmap_t(&tx, X, TmType::kBf16, K, T, K, 64, 8 * nt, true))
     return QLORA_ERR_CUDA;
-  const GvShape g = gv_shape(N, K, false);
+  const GvShape g = gv_shape(N, K);
   const int G = static_cast<int>(std::min<int64_t>(std::min<int64_t>(g.total, sms), kGvMaxCtas));
-  GvParams p = gv_params(T, N, K, g, G);
+  GvParams p = {};
+  p.T = static_cast<int>(T);
+  p.rows = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.spt = g.spt;
+  p.tiles = g.tiles;
+  p.total = g.total;
+  p.maxseg = gv_maxseg(g, G);
   p.kbw = static_cast<int>(K / 64);
   p.e4m3 = W->absmax_e4m3;
   p.s2 = W->scale2;
@@ -468,12 +471,16 @@ int gemv_fwd(const void* X, int64_t T, const qlora_nf4_tensor* W, const void* B,
   p.sU = static_cast<const __nv_bfloat16*>(sU);
   p.Bw = static_cast<const __nv_bfloat16*>(B);
   p.r = r;
-  p.out_scale = 1.0f;
   p.out = static_cast<__nv_bfloat16*>(Y);
   p.ldo = N;
   p.part = reinterpret_cast<float*>(gws + L.part_w);
   p.ticket = reinterpret_cast<unsigned*>(gws + L.ticket_w);
-  return launch_gemv<false>(nt, ta, tx, p, G, true, st);
+  switch (nt) {
+    case 1: return launch_gemv_nt<1>(ta, tx, p, G, st);
+    case 2: return launch_gemv_nt<2>(ta, tx, p, G, st);
+    case 4: return launch_gemv_nt<4>(ta, tx, p, G, st);
+    default: return launch_gemv_nt<8>(ta, tx, p, G, st);
+  }
 }
 
 int compute_sU(const void* X, int64_t T, int64_t K, const void* A, int r, float s, void* sU, float* part,
