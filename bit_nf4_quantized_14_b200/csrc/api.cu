@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <climits>
 #include <atomic>
 #include <cstring>
 #include <mutex>
@@ -242,16 +243,26 @@ int launch_nf4_linear(const void* act, int64_t T, const qlora_nf4_tensor* W, con
   return launched();
 }
 
+// The adapter GEMMs stream X or dY once: a ring of about 96 KB keeps two CTAs on every SM.
 template <int BN> constexpr int skinny_stages() {
   constexpr int stage = 128 * 64 * 2 + BN * 64 * 2;
-  return std::min(6, (200 * 1024) / stage);
+  return std::max(2, std::min(6, (96 * 1024) / stage));
 }
 
+// Split of the contraction: the number of slices s (each at least 4 blocks) that minimises
+// waves(s) * (blocks per slice + 4), waves counted against kTargetCtas resident CTAs (two per SM of a
+// B200), so that the grid fills whole waves instead of leaving a short last one; the +4 charges each
+// slice its pipeline fill and its partial-sum write.
 struct Split { int splits, kb_split; };
 Split choose_split(int64_t tiles, int64_t nkb) {
-  int64_t want = std::max<int64_t>(1, cdiv(kTargetCtas, tiles));
-  want = std::min<int64_t>(want, std::max<int64_t>(1, nkb / 4));
-  const int64_t kb_split = cdiv(nkb, want);
+  const int64_t max_s = std::max<int64_t>(1, nkb / 4);
+  int64_t best_s = 1, best_cost = INT64_MAX;
+  for (int64_t s = 1; s <= max_s; ++s) {
+    const int64_t kb = cdiv(nkb, s), real_s = cdiv(nkb, kb);
+    const int64_t cost = cdiv(tiles * real_s, kTargetCtas) * (kb + 4);   // + pipeline fill and partials
+    if (cost < best_cost) { best_cost = cost; best_s = real_s; }
+  }
+  const int64_t kb_split = cdiv(nkb, best_s);
   return {static_cast<int>(cdiv(nkb, kb_split)), static_cast<int>(kb_split)};
 }
 
