@@ -548,8 +548,17 @@ def run_codec_sweep(args):
         ms = time_calls(lambda: q.dequantize(out, torch.bfloat16, out=deq), flush, args.steps, args.warmup)
         row["dequantize_bf16"] = {"us": round(ms * 1e3, 2), "GB/s": round(n * DEQ_B_PER_ELEM / (ms / 1e3) / 1e9, 1),
                                   "frac": round(n * DEQ_B_PER_ELEM / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
+        # the variant without double quantization: fp32 constants, 0.5 + 4/64 B per element stored
+        single = q.NF4SingleWeight.empty(1, n, device)
+        sb = 0.5 + 4 / 64
+        for name, fn, bpe in (("quantize_single_fp32", lambda: q.quantize_single(x[:n].view(1, n), out=single), 4 + sb),
+                              ("dequantize_single_bf16", lambda: q.dequantize_single(single, torch.bfloat16, out=deq),
+                               sb + 2)):
+            ms = time_calls(fn, flush, args.steps, args.warmup)
+            row[name] = {"us": round(ms * 1e3, 2), "GB/s": round(n * bpe / (ms / 1e3) / 1e9, 1),
+                         "frac": round(n * bpe / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
         cases.append(row)
-        del out, ws, deq
+        del out, ws, deq, single
     status = q.get_status()
     top = cases[-1]
     print(json.dumps({"metric": "NF4 quantize / dequantize HBM GB/s over the size sweep (value: fp32 quantize "

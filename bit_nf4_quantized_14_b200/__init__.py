@@ -66,6 +66,8 @@ def _open() -> ctypes.CDLL:
         "qlora_nf4_quantize": [vp, i32, i64, i64, P(_NF4Struct), vp, sz, vp],
         "qlora_nf4_quantize_noalloc": [vp, i32, i64, i64, P(_NF4Struct), vp],
         "qlora_nf4_dequantize": [P(_NF4Struct), vp, i32, vp],
+        "qlora_nf4_quantize_single": [vp, i32, i64, i64, vp, vp, vp],
+        "qlora_nf4_dequantize_single": [vp, vp, i64, i64, vp, i32, vp],
         "qlora_linear_workspace": [i64, i64, i64, i32, P(sz)],
         "qlora_linear_fwd": [vp, i64, P(_NF4Struct), vp, vp, i32, ctypes.c_float, vp, vp, vp, sz, vp],
         "qlora_linear_bwd": [vp, vp, i64, P(_NF4Struct), vp, vp, i32, ctypes.c_float, vp, vp, vp, vp,
@@ -179,6 +181,46 @@ def quantize(w: torch.Tensor, out: NF4Weight | None = None, workspace: torch.Ten
     _check(load().qlora_nf4_quantize(_ptr(w), QLORA_F32 if w.dtype == torch.float32 else QLORA_BF16, rows, cols,
                                   ctypes.byref(st), _ptr(ws), ws.numel(), _stream(stream)), "qlora_nf4_quantize")
     return q
+
+
+@dataclass
+class NF4SingleWeight:
+    """NF4 codes with the fp32 block constants kept per block of 64 (no double quantization)."""
+    codes: torch.Tensor      # uint8[ceil(n/2)]
+    absmax: torch.Tensor     # float32[ceil(n/64)]
+    rows: int
+    cols: int
+
+    @classmethod
+    def empty(cls, rows: int, cols: int, device) -> "NF4SingleWeight":
+        n = rows * cols
+        return cls(torch.empty(-(-n // 2), dtype=torch.uint8, device=device),
+                   torch.empty(-(-n // 64), dtype=torch.float32, device=device), rows, cols)
+
+
+def quantize_single(w: torch.Tensor, out: NF4SingleWeight | None = None, stream=None) -> NF4SingleWeight:
+    """NF4 codes + fp32 block constants of a CUDA fp32 or bf16 tensor (1-D or 2-D, contiguous)."""
+    if w.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("quantize_single: w must be float32 or bfloat16")
+    _need(w, w.dtype, "w")
+    rows, cols = (w.shape[0], w.shape[1]) if w.dim() == 2 else (1, w.numel())
+    q = out if out is not None else NF4SingleWeight.empty(rows, cols, w.device)
+    _check(load().qlora_nf4_quantize_single(_ptr(w), QLORA_F32 if w.dtype == torch.float32 else QLORA_BF16, rows,
+                                            cols, _ptr(q.codes), _ptr(q.absmax), _stream(stream)),
+           "qlora_nf4_quantize_single")
+    return q
+
+
+def dequantize_single(q: NF4SingleWeight, dtype=torch.bfloat16, out: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    if dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("dequantize_single: dtype must be float32 or bfloat16")
+    o = out if out is not None else torch.empty(q.rows, q.cols, dtype=dtype, device=q.codes.device)
+    _need(o, dtype, "out")
+    _check(load().qlora_nf4_dequantize_single(_ptr(q.codes), _ptr(q.absmax), q.rows, q.cols, _ptr(o),
+                                              QLORA_F32 if dtype == torch.float32 else QLORA_BF16, _stream(stream)),
+           "qlora_nf4_dequantize_single")
+    return o
 
 
 NOALLOC_MAX_NUMEL = 1 << 26

@@ -570,6 +570,22 @@ int run_quantize(const void* w, int w_dtype, int64_t n, const qlora_nf4_tensor* 
     return QLORA_ERR_CUDA;
   return launched();
 }
+
+// The bulk-copy dequantizer in either constant format (double-quantized, or fp32 per block).
+int launch_dequant(bool bf16, bool single, const uint8_t* codes, const uint8_t* e4m3, const float* s2,
+                   const float* mu, const float* c1, int64_t n, void* out, int sms, cudaStream_t st) {
+  auto kern = bf16 ? (single ? nf4_dequantize_kernel<true, true> : nf4_dequantize_kernel<true, false>)
+                   : (single ? nf4_dequantize_kernel<false, true> : nf4_dequantize_kernel<false, false>);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDeqSmemBytes) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDeqThreads, kDeqSmemBytes) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(
+      std::max<int64_t>(1, std::min<int64_t>(cdiv(n, kGroupElems), int64_t(sms) * std::max(per_sm, 1))));
+  kern<<<grid, kDeqThreads, kDeqSmemBytes, st>>>(codes, e4m3, s2, mu, c1, n, out, codebook());
+  return launched();
+}
 }  // namespace
 }  // namespace qnf4
 
@@ -642,19 +658,47 @@ int qlora_nf4_dequantize(const qlora_nf4_tensor* q, void* out, int out_dtype, ql
   if (int e = check_device(&sms)) return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t n = q->rows * q->cols;
-  const bool bf16 = out_dtype == QLORA_BF16;
-  auto kern = bf16 ? nf4_dequantize_kernel<true> : nf4_dequantize_kernel<false>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDeqSmemBytes) != cudaSuccess)
-    return QLORA_ERR_CUDA;
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDeqThreads, kDeqSmemBytes) != cudaSuccess)
-    return QLORA_ERR_CUDA;
-  const unsigned grid = static_cast<unsigned>(
-      std::max<int64_t>(1, std::min<int64_t>(cdiv(n, kGroupElems), int64_t(sms) * std::max(per_sm, 1))));
   ProfScope prof(QLORA_PROF_DEQUANTIZE, st);
-  kern<<<grid, kDeqThreads, kDeqSmemBytes, st>>>(q->codes, q->absmax_e4m3, q->scale2, q->offset, n, out,
-                                                 codebook());
+  return launch_dequant(out_dtype == QLORA_BF16, false, q->codes, q->absmax_e4m3, q->scale2, q->offset, nullptr, n,
+                        out, sms, st);
+}
+
+int qlora_nf4_quantize_single(const void* w, int w_dtype, int64_t rows, int64_t cols, void* codes, float* absmax,
+                              qlora_stream_t stream) {
+  if (!w || !codes || !absmax) return QLORA_ERR_INVALID_ARG;
+  if (w_dtype != QLORA_F32 && w_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
+  if (rows <= 0 || cols <= 0 || rows > kMaxNumel / cols) return QLORA_ERR_SHAPE;
+  if (!aligned16(w) || !aligned16(codes) || !aligned16(absmax)) return QLORA_ERR_ALIGNMENT;
+  int sms = 0;
+  if (int e = check_device(&sms)) return e;
+  const Buckets& bk = buckets();
+  if (!bk.ok) return QLORA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t n = rows * cols, ns = cdiv(n, kSlabElems);
+  const unsigned g1 = static_cast<unsigned>(std::min<int64_t>(cdiv(ns, kQuantThreads / 32), int64_t(sms) * kQuantMinBlocks));
+  ProfScope prof(QLORA_PROF_QUANTIZE, st);
+  uint8_t* c = static_cast<uint8_t*>(codes);
+  if (w_dtype == QLORA_F32)
+    nf4_quantize_pass1<float><<<g1, kQuantThreads, 0, st>>>(static_cast<const float*>(w), n, c, absmax, nullptr, ns,
+                                                             codebook(), bk.arg, nullptr);
+  else
+    nf4_quantize_pass1<__nv_bfloat16><<<g1, kQuantThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(w), n, c,
+                                                                     absmax, nullptr, ns, codebook(), bk.arg, nullptr);
   return launched();
+}
+
+int qlora_nf4_dequantize_single(const void* codes, const float* absmax, int64_t rows, int64_t cols, void* out,
+                                int out_dtype, qlora_stream_t stream) {
+  if (!codes || !absmax || !out) return QLORA_ERR_INVALID_ARG;
+  if (out_dtype != QLORA_F32 && out_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
+  if (rows <= 0 || cols <= 0 || rows > kMaxNumel / cols) return QLORA_ERR_SHAPE;
+  if (!aligned16(codes) || !aligned16(absmax) || !aligned16(out)) return QLORA_ERR_ALIGNMENT;
+  int sms = 0;
+  if (int e = check_device(&sms)) return e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  ProfScope prof(QLORA_PROF_DEQUANTIZE, st);
+  return launch_dequant(out_dtype == QLORA_BF16, true, static_cast<const uint8_t*>(codes), nullptr, nullptr, nullptr,
+                        absmax, rows * cols, out, sms, st);
 }
 
 int qlora_linear_workspace(int64_t T, int64_t N, int64_t K, int r, size_t* bytes) {

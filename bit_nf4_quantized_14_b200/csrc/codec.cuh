@@ -163,13 +163,14 @@ __device__ __forceinline__ float block_codes(const float (&x)[16], float lotab, 
 // Pass 1. Each warp owns slabs gw, gw + nw, ... and walks them as a flat sequence of 8-block steps,
 // loading step i+1 while step i computes. Per slab it writes the 64 block constants (fp32) and their
 // fp64 balanced-tree sum. A ragged last slab is done by one warp at the end, with bounds on every element.
+// Without double quantization (ssum and ticket null) c1 is the stored constant array and pass 1 is all.
 template <typename InT>
 __global__ void __launch_bounds__(kQuantThreads, kQuantMinBlocks) nf4_quantize_pass1(
     const InT* __restrict__ w, int64_t n, uint8_t* __restrict__ codes, float* __restrict__ c1,
     double* __restrict__ ssum, int64_t nslabs, CodebookArg cb, BucketArg bk, unsigned* __restrict__ ticket) {
   __shared__ float c1buf[kQuantThreads / 32][kSlabBlocks];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0u;    // arrival counter of the mean pass
+  if (ticket && blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0u;    // arrival counter of the mean pass
   const float lotab = __uint_as_float((bk.lo_nibbles[lane >> 3] >> (4 * (lane & 7))) & 0xFu);
   const float ttab = (lane < 15) ? cb.thresholds[lane] : __int_as_float(0x7F800000);
   const int64_t nb = (n + kBlock - 1) / kBlock;
@@ -191,7 +192,7 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinBlocks) nf4_quantize_p
       const double r = __shfl_down_sync(0xffffffffu, t, off);
       if ((lane & (2 * off - 1)) == 0) t = t + r;    // left subtree + right subtree
     }
-    if (lane == 0) ssum[s] = t;
+    if (lane == 0 && ssum) ssum[s] = t;
     __syncwarp();
   };
 
@@ -400,18 +401,21 @@ __device__ __forceinline__ void store8(const float (&v)[8], void* __restrict__ o
 constexpr int kDeqThreads = 256;
 constexpr int kDeqStages = 8;
 constexpr uint32_t kDeqCodeBytes = kGroupElems / 2;
-constexpr uint32_t kDeqStageBytes = kDeqCodeBytes + kGroup;
-constexpr uint32_t kDeqSmemBytes = kDeqStages * kDeqStageBytes;
+constexpr uint32_t kDeqSmemBytes = kDeqStages * (kDeqCodeBytes + kGroup * 4);   // enough for either kind
 
-template <bool kBf16Out>
+// kSingle: the constants are stored as fp32 c1 per block (no second level); `c1` replaces e4m3/s2/mu.
+template <bool kBf16Out, bool kSingle>
 __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_kernel(
     const uint8_t* __restrict__ codes, const uint8_t* __restrict__ e4m3, const float* __restrict__ s2,
-    const float* __restrict__ mu_ptr, int64_t n, void* __restrict__ out, CodebookArg cb) {
+    const float* __restrict__ mu_ptr, const float* __restrict__ c1, int64_t n, void* __restrict__ out,
+    CodebookArg cb) {
+  constexpr uint32_t kConstBytes = kSingle ? kGroup * 4 : kGroup;
+  constexpr uint32_t kStageBytes = kDeqCodeBytes + kConstBytes;
   extern __shared__ __align__(128) unsigned char dsm[];
   __shared__ uint64_t bars[kDeqStages];
   const int tid = threadIdx.x, lane = tid & 31;
   const float qreg = cb.levels[lane & 15];
-  const float mu = *mu_ptr;
+  const float mu = kSingle ? 0.0f : *mu_ptr;
   const int64_t nfull = n / kGroupElems;
   const int64_t ngroups = (n + kGroupElems - 1) / kGroupElems;
   const int64_t my =
@@ -427,10 +431,11 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_kernel(
       const int64_t g = blockIdx.x + issued * gridDim.x;
       if (g >= nfull) continue;
       const int s = static_cast<int>(issued % kDeqStages);
-      unsigned char* st = dsm + s * kDeqStageBytes;
-      mbar_arrive_expect_tx(&bars[s], kDeqStageBytes);
+      unsigned char* st = dsm + s * kStageBytes;
+      mbar_arrive_expect_tx(&bars[s], kStageBytes);
       bulk_load(st, codes + g * kDeqCodeBytes, kDeqCodeBytes, &bars[s]);
-      bulk_load(st + kDeqCodeBytes, e4m3 + g * kGroup, kGroup, &bars[s]);
+      if constexpr (kSingle) bulk_load(st + kDeqCodeBytes, c1 + g * kGroup, kConstBytes, &bars[s]);
+      else bulk_load(st + kDeqCodeBytes, e4m3 + g * kGroup, kConstBytes, &bars[s]);
     }
   };
   if (tid == 0) issue_upto(kDeqStages);
@@ -438,18 +443,20 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_kernel(
   int timed_out = 0;
   for (; i < my; ++i) {
     const int64_t g = blockIdx.x + i * gridDim.x;
-    const float sg = s2[g];
+    const float sg = kSingle ? 0.0f : s2[g];
     if (g < nfull) {
       const int s = static_cast<int>(i % kDeqStages);
       if (!mbar_wait(&bars[s], static_cast<uint32_t>((i / kDeqStages) & 1))) timed_out = 1;
-      const unsigned char* st = dsm + s * kDeqStageBytes;
+      const unsigned char* st = dsm + s * kStageBytes;
       const uint32_t* cw = reinterpret_cast<const uint32_t*>(st);
       const uint8_t* ev = st + kDeqCodeBytes;
+      const float* cv = reinterpret_cast<const float*>(st + kDeqCodeBytes);
 #pragma unroll 4
       for (int k = 0; k < kGroupElems / 8 / kDeqThreads; ++k) {
         const int j = tid + kDeqThreads * k;           // chunk within the group; its block is j / 8
         float v[8];
-        dequant8(cw[j], __fmaf_rn(decode_e4m3(ev[j >> 3]), sg, mu), qreg, v);
+        const float sc = kSingle ? cv[j >> 3] : __fmaf_rn(decode_e4m3(ev[j >> 3]), sg, mu);
+        dequant8(cw[j], sc, qreg, v);
         store8<kBf16Out>(v, out, g * (kGroupElems / 8) + j);
       }
     } else {
@@ -459,7 +466,8 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_kernel(
         const int64_t c = cw0 + lane;                  // cw0 is the warp's first chunk: warp-uniform loop
         const bool ok = c < c_end;
         const uint32_t x = ok ? reinterpret_cast<const uint32_t*>(codes)[c] : 0u;
-        const float sc = ok ? __fmaf_rn(decode_e4m3(e4m3[(c * 8) / kBlock]), sg, mu) : 0.0f;
+        const int64_t blk = (c * 8) / kBlock;
+        const float sc = !ok ? 0.0f : kSingle ? c1[blk] : __fmaf_rn(decode_e4m3(e4m3[blk]), sg, mu);
         float v[8];
         dequant8(x, sc, qreg, v);
         if (ok) store8<kBf16Out>(v, out, c);
@@ -468,7 +476,8 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_kernel(
         for (int64_t e = c_end * 8; e < n; ++e) {
           const uint8_t byte = codes[e / 2];
           const uint32_t code = (e & 1) ? (byte & 0xFu) : (byte >> 4);
-          const float v = __fmul_rn(cb.levels[code], __fmaf_rn(decode_e4m3(e4m3[e / kBlock]), sg, mu));
+          const float sc = kSingle ? c1[e / kBlock] : __fmaf_rn(decode_e4m3(e4m3[e / kBlock]), sg, mu);
+          const float v = __fmul_rn(cb.levels[code], sc);
           if constexpr (kBf16Out) reinterpret_cast<__nv_bfloat16*>(out)[e] = __float2bfloat16_rn(v);
           else reinterpret_cast<float*>(out)[e] = v;
         }

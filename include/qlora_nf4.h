@@ -152,6 +152,22 @@ int qlora_nf4_quantize_noalloc(const void* w, int w_dtype, int64_t rows, int64_t
 int qlora_nf4_dequantize(const qlora_nf4_tensor* q, void* out, int out_dtype, qlora_stream_t stream);
 
 /*
+ * NF4 without double quantization: the same 4-bit codes (two per byte, even element in the high
+ * nibble) with the fp32 block constants kept as they are [PEFT "Double quantization": the constants
+ * before the second level, 32/64 = 0.5 bits per weight; "The real way": double quantization is one of
+ * the listed savings]. For an n-element tensor the caller allocates `codes` (ceil(n/2) bytes) and
+ * `absmax` (ceil(n/64) fp32), both device pointers, 16-byte aligned.
+ *   qlora_nf4_quantize_single writes both from w (rows x cols, QLORA_F32 or QLORA_BF16); codes are
+ *     identical to qlora_nf4_quantize's. A non-finite input sets QLORA_STATUS_NONFINITE. No workspace.
+ *   qlora_nf4_dequantize_single writes w_hat = fp32(level[code] * absmax[block]), rounded to bf16 (RNE)
+ *     for QLORA_BF16 output.
+ */
+int qlora_nf4_quantize_single(const void* w, int w_dtype, int64_t rows, int64_t cols, void* codes,
+                              float* absmax, qlora_stream_t stream);
+int qlora_nf4_dequantize_single(const void* codes, const float* absmax, int64_t rows, int64_t cols,
+                                void* out, int out_dtype, qlora_stream_t stream);
+
+/*
  * Device workspace bytes for qlora_linear_fwd / qlora_linear_bwd with T tokens, weight N x K (out x in)
  * and LoRA rank r (host output). One buffer of this size serves both calls.
  */

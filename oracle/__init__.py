@@ -28,7 +28,8 @@ from .lowp import (rn32_add, rn32_sub, rn32_mul, rn32_div, fma32, bf16_rne_bits,
                    e4m3_decode, e4m3_encode, E4M3_MAX)
 from .codec import (BLOCK, DQ_BLOCK, num_blocks, num_groups, storage_bytes, absmax_blocks,
                     nf4_codes, pack_codes, unpack_codes, pairwise_tree_sum, block_mean,
-                    double_quantize, double_dequantize, quantize, dequantize, NF4Tensor)
+                    double_quantize, double_dequantize, quantize, dequantize, NF4Tensor,
+                    quantize_single, dequantize_single, storage_bytes_single, NF4SingleTensor)
 from .linear import linear_fwd, linear_bwd
 
 __all__ = [n for n in dir() if not n.startswith("_")]

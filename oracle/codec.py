@@ -32,6 +32,10 @@ Readings where the pages leave a step open:
           block), s2 (fp32 per group) and mu (fp32).
   R-deq   c1_hat_b = fma(decode(e_b), s2_g, mu) with one rounding; w_hat = RN32(q[code] * c1_hat_b),
           then bf16 round-to-nearest-even for bf16 output.  No clamping of c1_hat.
+  R-single the variant without double quantization (PEFT page, "Double quantization": the fp32 block
+          constants as stored before the second level; "The real way" lists double quantization as an
+          option): the same codes, the fp32 c1 stored per block (0.5 bits/param of overhead), and
+          w_hat = RN32(q[code] * c1_b), bf16 round-to-nearest-even for bf16 output.
 """
 from __future__ import annotations
 
@@ -198,3 +202,44 @@ def dequantize(t: NF4Tensor, out: str = "bf16") -> np.ndarray:
     if out == "bf16":
         return bf16_rne_bits(w).reshape(t.shape)
     raise ValueError(out)
+
+
+# ---- the variant without double quantization (reading R-single) ------------------------------------
+
+@dataclass
+class NF4SingleTensor:
+    codes: np.ndarray        # uint8[ceil(n/2)], as in NF4Tensor
+    absmax: np.ndarray       # fp32[nb]: the block constants c1 themselves
+    n: int
+    shape: tuple
+
+
+def quantize_single(w, shape=None) -> NF4SingleTensor:
+    """NF4 codes with the fp32 block constants kept as they are (no second level)."""
+    w32 = as_f32_values(w)
+    _, T = nf4_codebook()
+    c1 = absmax_blocks(w32)
+    shp = tuple(np.asarray(w).shape) if shape is None else tuple(shape)
+    return NF4SingleTensor(pack_codes(nf4_codes(w32, c1, T)), c1.astype(np.float32), int(w32.size), shp)
+
+
+def dequantize_single(t: NF4SingleTensor, out: str = "bf16") -> np.ndarray:
+    """w_hat = RN32(q[code] * c1_b); bf16 output as uint16 bit patterns, fp32 as fp32."""
+    q, _ = nf4_codebook()
+    codes = unpack_codes(t.codes, t.n)
+    w = np.empty(t.n, dtype=np.float32)
+    for s in range(0, t.n, _CHUNK):
+        m = min(_CHUNK, t.n - s)
+        c1_e = np.repeat(t.absmax[s // BLOCK:(s + m + BLOCK - 1) // BLOCK], BLOCK)[:m]
+        w[s:s + m] = rn32_mul(q[codes[s:s + m]], c1_e)
+    if out == "f32":
+        return w.reshape(t.shape)
+    if out == "bf16":
+        return bf16_rne_bits(w).reshape(t.shape)
+    raise ValueError(out)
+
+
+def storage_bytes_single(n: int) -> dict:
+    """Bytes of each stored array of an n-element NF4 tensor with fp32 block constants."""
+    return {"codes": -(-n // 2), "absmax": 4 * num_blocks(n)}
+

@@ -194,3 +194,38 @@ def test_codes_over_every_bf16_value(lib, dtype):
     assert st == 0
     assert_same_as_oracle(q, ref)
     assert_dequant_same(lib, q, ref, x.shape)
+
+
+# ---- the variant without double quantization --------------------------------------------------
+
+def _assert_single_same(lib, x_dev, ref, n):
+    qs = lib.quantize_single(x_dev)
+    assert lib.get_status() == 0
+    assert np.array_equal(qs.codes.cpu().numpy(), ref.codes), "codes"
+    assert np.array_equal(qs.absmax.cpu().numpy().view(np.uint32), ref.absmax.view(np.uint32)), "fp32 constants"
+    got16 = lib.dequantize_single(qs, torch.bfloat16).cpu().view(torch.int16).numpy().view(np.uint16).reshape(-1)
+    assert np.array_equal(got16, O.dequantize_single(ref, "bf16").reshape(-1)), "bf16 dequant"
+    got32 = lib.dequantize_single(qs, torch.float32).cpu().numpy().reshape(-1)
+    assert np.array_equal(got32.view(np.uint32), O.dequantize_single(ref, "f32").reshape(-1).view(np.uint32))
+    return qs
+
+
+@pytest.mark.parametrize("n", [1, 63, 65, 4097, 16383, 16385, 3 * 16384 + 77, 64 * 256 * 37 + 5])
+def test_single_variant_ragged_sizes(lib, n):
+    x = synth.sweep_f32(n, seed=7, tensor_id=n % 997)
+    _assert_single_same(lib, torch.from_numpy(x.reshape(1, n)).cuda(), O.quantize_single(x), n)
+    xb = synth.to_bf16(x)
+    _assert_single_same(lib, xb.reshape(1, n).cuda(), O.quantize_single(synth.bf16_bits(xb)), n)
+
+
+def test_single_variant_codes_match_the_double_quantized_path(lib):
+    W = synth.weight_f32(1024, 4096, seed=3, tensor_id=2)
+    d = lib.quantize(torch.from_numpy(W).cuda())
+    s = _assert_single_same(lib, torch.from_numpy(W).cuda(), O.quantize_single(W), W.size)
+    assert torch.equal(d.codes, s.codes)
+
+
+def test_single_variant_special_values(lib):
+    x = np.concatenate([np.zeros(128, np.float32), np.float32([1e-40, -3e-39] + [0.0] * 62),
+                        np.float32([3e38, -1e38] + [1e30] * 62), synth.normal_f32(64 * 50 + 3, 0.02, 0, 77)])
+    _assert_single_same(lib, torch.from_numpy(x).cuda(), O.quantize_single(x), x.size)

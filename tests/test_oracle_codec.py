@@ -222,3 +222,46 @@ def test_codebook_statistics_match_the_page():
     _, rms_lloyd = run(lv)
     gain = 1 - rms_lloyd / rms_nf4
     assert abs(gain - GOLDEN["lloyd_gain_over_nf4"]["value"]) < 0.03, gain
+
+
+# ---- the variant without double quantization ---------------------------------------------------
+
+def test_single_variant_overhead_is_half_a_bit_per_weight():
+    """PEFT page, 'Double quantization': fp32 constants per block of 64 cost 32/64 = 0.5 bits/param."""
+    n = 64 * 4096
+    sb = O.storage_bytes_single(n)
+    assert 8.0 * sb["absmax"] / n == GOLDEN["overhead_bits_before_dq"]["value"]
+    assert sb["codes"] == n // 2
+
+
+def test_single_variant_shares_codes_and_dequantizes_by_definition():
+    x = synth.sweep_f32(64 * 300 + 17, seed=5, tensor_id=12)
+    s = O.quantize_single(x)
+    d = O.quantize(x)
+    assert np.array_equal(s.codes, d.codes)                        # the first level is unchanged
+    assert np.array_equal(s.absmax.view(np.uint32), O.absmax_blocks(x).view(np.uint32))
+    q, _ = O.nf4_codebook()
+    codes = O.unpack_codes(s.codes, s.n)
+    want = (q[codes].astype(np.float64) * np.repeat(s.absmax, 64)[:s.n].astype(np.float64)).astype(np.float32)
+    assert np.array_equal(O.dequantize_single(s, "f32").view(np.uint32), want.view(np.uint32))
+
+
+def test_single_and_double_agree_when_the_second_level_is_exact():
+    """All block constants equal: s2 = 0 and c1_hat = mu = c1 exactly, so both variants dequantize alike."""
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal(64 * 512) * 0.01).astype(np.float32)
+    x.reshape(-1, 64)[:, 0] = np.float32(0.25)                       # every block's absmax is 0.25
+    s, d = O.quantize_single(x), O.quantize(x)
+    assert np.all(d.scale2 == 0)
+    assert np.array_equal(O.dequantize_single(s, "bf16"), O.dequantize(d, "bf16"))
+
+
+def test_single_variant_error_bound():
+    """|w - w_hat| <= a * max_j (T_j - q_j) + fp32 rounding, per block (nearest-level quantization)."""
+    x = synth.sweep_f32(64 * 2000, seed=6, tensor_id=13)
+    s = O.quantize_single(x)
+    q, T = O.nf4_codebook()
+    half_gap = float(np.max(np.maximum(T - q[:-1], q[1:] - T)))
+    a = np.repeat(s.absmax, 64)[:s.n].astype(np.float64)
+    err = np.abs(O.dequantize_single(s, "f32").astype(np.float64) - x.astype(np.float64))
+    assert np.all(err <= a * half_gap * (1 + 1e-6) + 1e-30)
