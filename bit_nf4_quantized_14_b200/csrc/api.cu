@@ -331,7 +331,7 @@ int check_nf4(const qlora_nf4_tensor* q) {
 
 struct LinearWs { size_t sU, sV, scales, part, total; };
 // ---- small-token path (T <= kGvMaxTokens): the stream-K GEMV kernels ---------------------------
-constexpr int kGvMaxCtas = 256;          // grid cap of the NF4 GEMV (>= the SM count of any B200)
+constexpr int kGvMaxCtas = 512;          // grid cap of the NF4 GEMV (>= two CTAs per SM of any B200)
 constexpr int kGuMaxSlices = 32;         // contraction slices of the adapter projection
 inline int gv_nt(int64_t T) { return T <= 8 ? 1 : T <= 16 ? 2 : T <= 32 ? 4 : 8; }
 struct GvShape { int spt, tiles; int64_t total; };
@@ -466,7 +466,8 @@ int gemv_fwd(const void* X, int64_t T, const qlora_nf4_tensor* W, const void* B,
       !make_tmap_t(&tx, X, TmType::kBf16, K, T, K, 64, 8 * nt, true))
     return QLORA_ERR_CUDA;
   const GvShape g = gv_shape(N, K);
-  const int G = static_cast<int>(std::min<int64_t>(std::min<int64_t>(g.total, sms), kGvMaxCtas));
+  const int per_sm = nt <= 4 ? GvCfg<1>::CTAS_PER_SM : GvCfg<8>::CTAS_PER_SM;
+  const int G = static_cast<int>(std::min<int64_t>(std::min<int64_t>(g.total, int64_t(sms) * per_sm), kGvMaxCtas));
   GvParams p = {};
   p.T = static_cast<int>(T);
   p.rows = static_cast<int>(N);

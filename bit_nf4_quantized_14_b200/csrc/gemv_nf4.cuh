@@ -7,11 +7,12 @@
 // multiplied in 16-bit precision" (PEFT page, zerotofrontier.app/sft/peft, "Paged optimizers, and QLoRA
 // end to end"; dequantization fused into the matrix multiply: same page, "The real way"). Here the
 // dequantization never materialises a weight tile:
-//   * TMA streams tiles of 240 weight rows x 256 contraction elements (128 code bytes per row, 128-byte
+//   * TMA streams tiles of 112 weight rows x 256 contraction elements (128 code bytes per row, 128-byte
 //     swizzle) and the matching 64-wide boxes of X through a ring of stages;
 //   * each consumer warp owns 16 rows and builds the A fragments of mma.sync m16n8k16 (bf16, fp32
 //     accumulate) directly from code bytes: one byte permute and one shared-memory lookup per byte in a
-//     256-entry table of bf16 level pairs, replicated per lane so lookups never conflict;
+//     256-entry table of bf16 level pairs, replicated per lane so lookups never conflict; two CTAs share
+//     an SM (for T <= 32) so that two stage pipelines run out of step;
 //   * the block constant c1_hat = fma(decode(e4m3), s2, mu) multiplies the fp32 block accumulator once per
 //     64-element block: y += c1_hat * sum_k bf16(level[code_k]) * x_k.
 // The one difference from the fused GEMM's W_hat = bf16(level * c1_hat) is where the bf16 rounding falls
@@ -31,13 +32,13 @@
 
 namespace qnf4 {
 
-constexpr int kGvWarps = 15;                      // consumer warps, 16 rows each (16 warps per CTA)
+constexpr int kGvWarps = 7;                       // consumer warps, 16 rows each (8 warps per CTA)
 constexpr int kGvRows = 16 * kGvWarps;            // rows per tile
 constexpr int kGvThreads = 32 * (kGvWarps + 1);   // + one producer warp
 constexpr int kGvRowBytes = 128;                  // code bytes per row per stage (256 elements)
 constexpr int kGvStageK = 256;
 constexpr int kGvTileBytes = kGvRows * kGvRowBytes;
-constexpr int kGvLutBytes = 256 * 256;            // entry e: 32 lanes x 4 B at e * 256 (second half unused)
+constexpr int kGvLutBytes = 256 * 128;            // entry e: 32 lanes x 4 B at e * 128
 constexpr int kGvMaxTokens = 64;
 
 template <int NT>
@@ -45,7 +46,8 @@ struct GvCfg {
   static constexpr int TP = 8 * NT;                          // tokens padded to the MMA's n8 tiles
   static constexpr int X_BOX = TP * 128;                     // one 64-wide box of X
   static constexpr int STAGE_BYTES = kGvTileBytes + 4 * X_BOX;
-  static constexpr int AVAIL = 227 * 1024 - 1024 - 256 - kGvLutBytes;
+  static constexpr int CTAS_PER_SM = NT <= 4 ? 2 : 1;          // two independent pipelines per SM
+  static constexpr int AVAIL = (227 / CTAS_PER_SM) * 1024 - 1024 - 256 - kGvLutBytes;
   static constexpr int STAGES = (AVAIL / STAGE_BYTES) < 8 ? (AVAIL / STAGE_BYTES) : 8;
   static constexpr int SMEM_BYTES = 1024 + kGvLutBytes + STAGES * STAGE_BYTES + 256;
   static constexpr int SLOT = kGvWarps * 32 * NT * 4;          // floats of one CTA's partial tile
@@ -105,12 +107,11 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
   return v;
 }
-// A fragment register of one code byte: the pair (level[hi nibble], level[lo nibble]) as bf16. The byte
-// permute builds the table offset byte * 256 + lane * 4 in one instruction (lane4 = lane * 4 in byte 0;
-// `byte` picks the code byte of w).
+// A fragment register of one code byte: the pair (level[hi nibble], level[lo nibble]) as bf16, from the
+// lane's own copy of the table (entry byte at byte * 128 + lane * 4; lut_lane includes lane * 4).
 template <int kByte>
-__device__ __forceinline__ uint32_t lut_pair(uint32_t lut, uint32_t w, uint32_t lane4) {
-  return lds32(lut + __byte_perm(w, lane4, 0x5504u | (kByte << 4)));
+__device__ __forceinline__ uint32_t lut_pair(uint32_t lut_lane, uint32_t w) {
+  return lds32(lut_lane + (__byte_perm(w, 0u, 0x4440u | kByte) << 7));
 }
 __device__ __forceinline__ uint32_t ldg32_or0(const __nv_bfloat16* p, bool ok) {
   return ok ? __ldg(reinterpret_cast<const unsigned int*>(p)) : 0u;
@@ -135,7 +136,7 @@ struct GvConsts {
 };
 
 template <int NT>
-__global__ void __launch_bounds__(kGvThreads, 1)
+__global__ void __launch_bounds__(kGvThreads, GvCfg<NT>::CTAS_PER_SM)
     nf4_gemv_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmX,
                     const GvParams p, const CodebookArg cb) {
   using C = GvCfg<NT>;
@@ -158,10 +159,10 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     }
     fence_barrier_init();
   }
-  // lut[e * 64 + l] = bf16 pair (level[e >> 4], level[e & 15]), one copy per lane l < 32
+  // lut[e * 32 + l] = bf16 pair (level[e >> 4], level[e & 15]), one copy per lane l
   for (int i = threadIdx.x; i < 256 * 32; i += kGvThreads) {
     const int e = i >> 5;
-    lut[e * 64 + (i & 31)] = pack_bf16x2(cb.levels[e >> 4], cb.levels[e & 15]);
+    lut[e * 32 + (i & 31)] = pack_bf16x2(cb.levels[e >> 4], cb.levels[e & 15]);
   }
   __syncthreads();
 
@@ -195,7 +196,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   // same permutation for A and for X, so the sum is unchanged. Lane j then needs bytes 8j .. 8j+7 of a
   // row's 32 code bytes (one 8-byte load) and elements 16j .. 16j+15 of a token's 64 (two 16-byte loads).
   const int g = lane >> 2, j = lane & 3;
-  const uint32_t lut_s = smem_u32(lut), lane4 = 4u * lane;
+  const uint32_t lut_lane = smem_u32(lut) + 4u * lane;
   const int rl0 = 16 * warp + g;                                   // tile-local rows of this thread
   const float mu = *p.mu;
   float acc[NT][4];
@@ -238,14 +239,14 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       const uint2 u0 = lds64(rowA0 + cc), u1 = lds64(rowA1 + cc);
       // A fragments per k16 step s: code byte 2s (elements 16j+4s, +1) and 2s+1 (+2, +3) of the 8
       uint32_t a[4][4];
-      a[0][0] = lut_pair<0>(lut_s, u0.x, lane4); a[0][2] = lut_pair<1>(lut_s, u0.x, lane4);
-      a[1][0] = lut_pair<2>(lut_s, u0.x, lane4); a[1][2] = lut_pair<3>(lut_s, u0.x, lane4);
-      a[2][0] = lut_pair<0>(lut_s, u0.y, lane4); a[2][2] = lut_pair<1>(lut_s, u0.y, lane4);
-      a[3][0] = lut_pair<2>(lut_s, u0.y, lane4); a[3][2] = lut_pair<3>(lut_s, u0.y, lane4);
-      a[0][1] = lut_pair<0>(lut_s, u1.x, lane4); a[0][3] = lut_pair<1>(lut_s, u1.x, lane4);
-      a[1][1] = lut_pair<2>(lut_s, u1.x, lane4); a[1][3] = lut_pair<3>(lut_s, u1.x, lane4);
-      a[2][1] = lut_pair<0>(lut_s, u1.y, lane4); a[2][3] = lut_pair<1>(lut_s, u1.y, lane4);
-      a[3][1] = lut_pair<2>(lut_s, u1.y, lane4); a[3][3] = lut_pair<3>(lut_s, u1.y, lane4);
+      a[0][0] = lut_pair<0>(lut_lane, u0.x); a[0][2] = lut_pair<1>(lut_lane, u0.x);
+      a[1][0] = lut_pair<2>(lut_lane, u0.x); a[1][2] = lut_pair<3>(lut_lane, u0.x);
+      a[2][0] = lut_pair<0>(lut_lane, u0.y); a[2][2] = lut_pair<1>(lut_lane, u0.y);
+      a[3][0] = lut_pair<2>(lut_lane, u0.y); a[3][2] = lut_pair<3>(lut_lane, u0.y);
+      a[0][1] = lut_pair<0>(lut_lane, u1.x); a[0][3] = lut_pair<1>(lut_lane, u1.x);
+      a[1][1] = lut_pair<2>(lut_lane, u1.x); a[1][3] = lut_pair<3>(lut_lane, u1.x);
+      a[2][1] = lut_pair<0>(lut_lane, u1.y); a[2][3] = lut_pair<1>(lut_lane, u1.y);
+      a[3][1] = lut_pair<2>(lut_lane, u1.y); a[3][3] = lut_pair<3>(lut_lane, u1.y);
       const uint32_t cX0 = static_cast<uint32_t>((2 * j) ^ g) << 4, cX1 = static_cast<uint32_t>((2 * j + 1) ^ g) << 4;
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
