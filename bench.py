@@ -663,6 +663,123 @@ def run_llama65b(args):
     return 0
 
 
+LLAMA65B_TRAIN_WORKLOAD = ("LLaMA-65B-shaped QLoRA training step: token embedding, 80 decoder layers (RMSNorm, causal "
+                           "attention with 64 heads over NF4+LoRA q/k/v/o, RMSNorm, SwiGLU over NF4+LoRA gate/up/"
+                           "down), final RMSNorm, bf16 output head, cross-entropy on uniform random targets, AdamW "
+                           "on the fp32 LoRA adapters (r = 64, alpha = 16); batch 1 x 512 tokens, vocab 32000, "
+                           "random init")
+
+
+def build_decoder(layers, d, ffn, heads, vocab, r, gen, device):
+    """A LLaMA-shaped decoder whose seven linears per layer are QLoRALinear modules (random init)."""
+    import torch
+    from bit_nf4_quantized_14_b200.autograd import QLoRALinear
+
+    def lin(n, k):
+        w = torch.randn(n, k, device=device, generator=gen).mul_(0.02)
+        m = QLoRALinear(w, r=r, alpha=ALPHA, generator=gen)
+        del w
+        return m
+
+    class Layer(torch.nn.Module):
+        def __init__(self):
+            super().__init__()
+            self.q, self.k, self.v, self.o = lin(d, d), lin(d, d), lin(d, d), lin(d, d)
+            self.gate, self.up, self.down = lin(ffn, d), lin(ffn, d), lin(d, ffn)
+            self.n1 = torch.ones(d, device=device, dtype=torch.bfloat16)
+            self.n2 = torch.ones(d, device=device, dtype=torch.bfloat16)
+
+        def forward(self, h):
+            T = h.shape[0]
+            x = rms(h, self.n1)
+            q = self.q(x).view(T, heads, d // heads).transpose(0, 1)
+            k = self.k(x).view(T, heads, d // heads).transpose(0, 1)
+            v = self.v(x).view(T, heads, d // heads).transpose(0, 1)
+            a = torch.nn.functional.scaled_dot_product_attention(q[None], k[None], v[None], is_causal=True)[0]
+            h = h + self.o(a.transpose(0, 1).reshape(T, d))
+            x = rms(h, self.n2)
+            return h + self.down(torch.nn.functional.silu(self.gate(x)) * self.up(x))
+
+    def rms(x, w, eps=1e-5):
+        xf = x.float()
+        return (xf * torch.rsqrt(xf.pow(2).mean(-1, keepdim=True) + eps)).to(torch.bfloat16) * w
+
+    class Decoder(torch.nn.Module):
+        def __init__(self):
+            super().__init__()
+            self.emb = (torch.randn(vocab, d, device=device, generator=gen) * 0.02).to(torch.bfloat16)
+            self.layers = torch.nn.ModuleList([Layer() for _ in range(layers)])
+            self.nf = torch.ones(d, device=device, dtype=torch.bfloat16)
+            self.head = (torch.randn(vocab, d, device=device, generator=gen) * 0.02).to(torch.bfloat16)
+
+        def forward(self, ids, targets):
+            h = self.emb[ids]
+            for layer in self.layers:
+                h = layer(h)
+            logits = rms(h, self.nf) @ self.head.t()
+            return torch.nn.functional.cross_entropy(logits.float(), targets)
+
+    return Decoder()
+
+
+def run_llama65b_train(args):
+    import torch
+    import bit_nf4_quantized_14_b200 as q
+    device = torch.device("cuda", 0)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(66)
+    vocab, T = 32000, LLAMA65B_TOKENS
+    model = build_decoder(LLAMA65B_LAYERS, 8192, 22016, 64, vocab, RANK_R, gen, device)
+    params = [p for p in model.parameters() if p.requires_grad]
+    opt = torch.optim.AdamW(params, lr=2e-4, weight_decay=0.0, fused=True)
+    ids = torch.randint(0, vocab, (T,), device=device, generator=gen)
+    targets = torch.randint(0, vocab, (T,), device=device, generator=gen)
+
+    def step():
+        loss = model(ids, targets)
+        loss.backward()
+        opt.step()
+        opt.zero_grad(set_to_none=True)
+        return loss
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    q.profile_read()
+    q.profile_enable(True)
+    clocks = ClockSampler(0)
+    clocks.start()
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = q.kernel_launches()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        loss = step()
+    ev1.record(stream)
+    while not ev1.query():
+        time.sleep(0.0005)
+    torch.cuda.synchronize()
+    launches = q.kernel_launches() - n0
+    clk = clocks.stop()
+    q.profile_enable(False)
+    prof = q.profile_read()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    lin_ms = sum(prof[c][1] for c in ("fwd_gemm", "bwd_gemm", "lora")) / args.steps
+    n_lora = sum(p.numel() for p in params)
+    print(json.dumps({"metric": "QLoRA training step, LLaMA-65B-shaped, tokens/s",
+                      "value": round(T / (ms / 1e3), 1), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+                      "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+                      "dtype": "bf16 (NF4 weights, fp32 adapters)", "data": "synthetic (random init, random ids)",
+                      "config": {"workload": LLAMA65B_TRAIN_WORKLOAD, "tokens": T, "r": RANK_R, "alpha": ALPHA,
+                                 "lora_params": n_lora, "nf4_weight_bytes": sum(
+                                     m.w.nbytes for m in model.modules() if hasattr(m, "w"))},
+                      "library_linears_ms_per_step": round(lin_ms, 3),
+                      "library_linears_share": round(lin_ms / ms, 4),
+                      "final_loss": float(loss.item()), "gpu_launches": int(launches), "clocks": clk,
+                      "device_status": q.get_status()}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -671,7 +788,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) measurement")
-    ap.add_argument("--workload", choices=["llama7b_step", "decode", "codec_sweep", "llama65b_linears"],
+    ap.add_argument("--workload", choices=["llama7b_step", "decode", "codec_sweep", "llama65b_linears",
+                                           "llama65b_train"],
                     default="llama7b_step",
                     help="llama7b_step (the headline line), or the decode / codec-sweep / 65B-step measurement lines")
     ap.add_argument("--shapes", default="all",
@@ -690,6 +808,8 @@ def main(argv=None):
         return run_codec_sweep(args)
     if args.workload == "llama65b_linears":
         return run_llama65b(args)
+    if args.workload == "llama65b_train":
+        return run_llama65b_train(args)
     return run_gpu(args)
 
 

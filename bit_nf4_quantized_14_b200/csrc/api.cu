@@ -5,6 +5,8 @@
 
 #include <algorithm>
 #include <climits>
+#include <cstdio>
+#include <cstdlib>
 #include <atomic>
 #include <cstring>
 #include <mutex>
@@ -25,10 +27,21 @@ constexpr int64_t kMaxNumel = int64_t(1) << 40;
 constexpr int64_t kMaxTokens = int64_t(65535) * 128;   // grid.y limit of the 128-row tiles
 constexpr int kTargetCtas = 2 * 148;                    // split heuristic: two waves of a B200
 std::atomic<int64_t> g_launches{0};
-inline int launched(int n = 1) {
-  g_launches.fetch_add(n, std::memory_order_relaxed);
-  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+// With QLORA_DEBUG set in the environment, a failed CUDA call is described on stderr (where and why).
+inline bool debug_on() {
+  static const bool on = std::getenv("QLORA_DEBUG") != nullptr;
+  return on;
 }
+inline int cuda_fail(cudaError_t e, const char* what, int line) {
+  if (debug_on()) std::fprintf(stderr, "qlora: %s failed at api.cu:%d: %s\n", what, line, cudaGetErrorString(e));
+  return QLORA_ERR_CUDA;
+}
+inline int launched_at(int line) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? QLORA_OK : cuda_fail(e, "kernel launch", line);
+}
+#define launched() launched_at(__LINE__)
 
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -104,13 +117,22 @@ QuantWs quant_ws(int64_t n) {
 }
 
 // ---- device checks ------------------------------------------------------------------------------
+// Also clears this host thread's pending non-sticky runtime error (cudaGetLastError is per thread, and a
+// caller's own earlier query -- an event or stream poll returning cudaErrorNotReady, for instance -- would
+// otherwise be reported as a failure of the launches that follow). A sticky error from a device fault is
+// returned again by every later call, so it is not hidden.
+// It also makes the device's primary context current on the calling thread (cudaSetDevice does so since
+// CUDA 12): the tensor maps are encoded through the driver API, which needs a current context, and a
+// thread that has made no runtime call yet -- PyTorch's autograd worker, for one -- has none.
 int check_device(int* num_sms) {
+  (void)cudaGetLastError();
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess)
+    return cuda_fail(cudaGetLastError(), "cudaGetDevice / cudaSetDevice", __LINE__);
   int major = 0, sms = 0;
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return QLORA_ERR_CUDA;
+    return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
   if (major != 10) return QLORA_ERR_UNSUPPORTED;
   if (num_sms) *num_sms = sms;
   return QLORA_OK;
@@ -168,6 +190,10 @@ bool make_tmap_t(CUtensorMap* m, const void* ptr, TmType t, uint64_t inner, uint
   const CUresult r = fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS && debug_on())
+    std::fprintf(stderr, "qlora: tensor map (ptr %p, dims %llu x %llu, stride %llu B, box %u x %u, swizzle %d) -> %d\n",
+                 ptr, (unsigned long long)inner, (unsigned long long)outer, (unsigned long long)(pitch * esz),
+                 box_inner, box_outer, (int)swizzle128, (int)r);
   return r == CUDA_SUCCESS;
 }
 bool make_tmap(CUtensorMap* m, const void* ptr, bool bf16, uint64_t inner, uint64_t outer,
@@ -189,7 +215,7 @@ int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUt
                 const CUtensorMap& b2, const GemmParams& p, cudaStream_t st) {
   auto kern = gemm_sm100_kernel<C>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
-    return QLORA_ERR_CUDA;
+    return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
   kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, a2, b2, p, codebook());
   return launched();
 }
@@ -226,7 +252,7 @@ int launch_nf4_linear(const void* act, int64_t T, const qlora_nf4_tensor* W, con
   else
     ok = ok && make_tmap(&tc, W->codes, false, K / 2, N, 64, 64) &&
          make_tmap_t(&tk, scales, TmType::kF32, kb_w, N, ld, 4, 64, false);
-  if (!ok) return QLORA_ERR_CUDA;
+  if (!ok) return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
   NF4GemmParams p{};
   p.T = static_cast<int>(T); p.F = static_cast<int>(F);
   p.nkb = static_cast<int>(cdiv(Cn, 64)); p.nkb2 = static_cast<int>(cdiv(r, 64));
@@ -237,7 +263,7 @@ int launch_nf4_linear(const void* act, int64_t T, const qlora_nf4_tensor* W, con
   p.lora_w = static_cast<const __nv_bfloat16*>(lora_w);
   auto kern = nf4_linear_gemm_kernel<Cfg>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
-    return QLORA_ERR_CUDA;
+    return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(p.num_tiles, sms));
   kern<<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, st>>>(tx, tc, tk, tuv, to, p, codebook());
   return launched();
@@ -414,7 +440,7 @@ int launch_gemv_nt(const CUtensorMap& ta, const CUtensorMap& tx, const GvParams&
   using C = GvCfg<NT>;
   auto kern = nf4_gemv_kernel<NT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
-    return QLORA_ERR_CUDA;
+    return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGvThreads);
@@ -425,14 +451,14 @@ int launch_gemv_nt(const CUtensorMap& ta, const CUtensorMap& tx, const GvParams&
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, ta, tx, p, codebook()) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tx, p, codebook()) != cudaSuccess) return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
   return launched();
 }
 
 // sU = s * X A^T for T <= kGvMaxTokens; clears both ticket arrays of the small-token path first.
 int gemv_sU(const void* X, int64_t T, int64_t K, const void* A, int r, float s, void* sU, char* gws,
             const GemvWs& L, cudaStream_t st) {
-  if (cudaMemsetAsync(gws + L.ticket_w, 0, L.ticket_bytes, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (cudaMemsetAsync(gws + L.ticket_w, 0, L.ticket_bytes, st) != cudaSuccess) return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
   const GuShape u = gu_shape(K, r);
   GuParams p = {};
   p.T = static_cast<int>(T);
@@ -464,7 +490,7 @@ int gemv_fwd(const void* X, int64_t T, const qlora_nf4_tensor* W, const void* B,
   CUtensorMap ta, tx;
   if (!make_tmap_t(&ta, W->codes, TmType::kU8, K / 2, N, K / 2, kGvRowBytes, kGvRows, true) ||
       !make_tmap_t(&tx, X, TmType::kBf16, K, T, K, 64, 8 * nt, true))
-    return QLORA_ERR_CUDA;
+    return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
   const GvShape g = gv_shape(N, K);
   const int per_sm = nt <= 4 ? GvCfg<1>::CTAS_PER_SM : GvCfg<8>::CTAS_PER_SM;
   const int G = static_cast<int>(std::min<int64_t>(std::min<int64_t>(g.total, int64_t(sms) * per_sm), kGvMaxCtas));
@@ -499,7 +525,7 @@ int compute_sU(const void* X, int64_t T, int64_t K, const void* A, int r, float 
                cudaStream_t st) {
   const int bn = static_cast<int>(cdiv(r, 64) * 64);
   CUtensorMap ta, tb;
-  if (!tmap_kmajor(&ta, X, K, T, 128) || !tmap_kmajor(&tb, A, K, r, bn)) return QLORA_ERR_CUDA;
+  if (!tmap_kmajor(&ta, X, K, T, 128) || !tmap_kmajor(&tb, A, K, r, bn)) return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
   const int64_t stride = cdiv(T, 128) * 128 * bn;
   if (int e = launch_skinny_bn<Skinny::kU>(bn, ta, tb, T, K, part, stride, st)) return e;
   return reduce_after(part, T, K, r, bn, s, sU, Red::kRowsBf16, st);
@@ -527,12 +553,12 @@ namespace {
 // Device address of this device's scratch array (set-up on the first call per device).
 int noalloc_scratch(void** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
   if (dev < 0 || dev >= kMaxDevices) return QLORA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> g(g_noalloc_mu);
   if (!g_noalloc_dev_ptr[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return QLORA_ERR_CUDA;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
     g_noalloc_dev_ptr[dev] = p;
   }
   *out = g_noalloc_dev_ptr[dev];
@@ -564,11 +590,11 @@ int run_quantize(const void* w, int w_dtype, int64_t n, const qlora_nf4_tensor* 
   if (int e = launched()) return e;
   if (launch_pdl(nf4_mean, L.mean_ctas, kTreeThreads, st, ssum, L.nslabs, nb, partial, ticket, out->offset) !=
       cudaSuccess)
-    return QLORA_ERR_CUDA;
+    return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
   if (int e = launched()) return e;
   if (launch_pdl(nf4_dq_pass2, static_cast<unsigned>(cdiv(ng, 8)), 256u, st, c1, nb, out->offset,
                  out->absmax_e4m3, out->scale2, ng) != cudaSuccess)
-    return QLORA_ERR_CUDA;
+    return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
   return launched();
 }
 
@@ -578,10 +604,10 @@ int launch_dequant(bool bf16, bool single, const uint8_t* codes, const uint8_t* 
   auto kern = bf16 ? (single ? nf4_dequantize_kernel<true, true> : nf4_dequantize_kernel<true, false>)
                    : (single ? nf4_dequantize_kernel<false, true> : nf4_dequantize_kernel<false, false>);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDeqSmemBytes) != cudaSuccess)
-    return QLORA_ERR_CUDA;
+    return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDeqThreads, kDeqSmemBytes) != cudaSuccess)
-    return QLORA_ERR_CUDA;
+    return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
   const unsigned grid = static_cast<unsigned>(
       std::max<int64_t>(1, std::min<int64_t>(cdiv(n, kGroupElems), int64_t(sms) * std::max(per_sm, 1))));
   kern<<<grid, kDeqThreads, kDeqSmemBytes, st>>>(codes, e4m3, s2, mu, c1, n, out, codebook());
@@ -772,7 +798,7 @@ int qlora_linear_bwd(const void* dY, const void* X, int64_t T, const qlora_nf4_t
     }
     // sV = s * dY B  (T x r): contraction over the N output features; B is N x r, i.e. MN-major.
     CUtensorMap tdy, tbl;
-    if (!tmap_kmajor(&tdy, dY, N, T, 128) || !tmap_mnmajor(&tbl, B, r, N)) return QLORA_ERR_CUDA;
+    if (!tmap_kmajor(&tdy, dY, N, T, 128) || !tmap_mnmajor(&tbl, B, r, N)) return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
     if (int e = launch_skinny_bn<Skinny::kV>(bn, tdy, tbl, T, N, part, cdiv(T, 128) * 128 * bn, st)) return e;
     if (int e = reduce_after(part, T, N, r, bn, s, sV, Red::kRowsBf16, st)) return e;
   }
@@ -784,14 +810,14 @@ int qlora_linear_bwd(const void* dY, const void* X, int64_t T, const qlora_nf4_t
   {
     // dA^T[k][j] = sum_t X[t][k] sV[t][j]  -> dA (r x K), transposed in the reduction
     CUtensorMap tx, tv;
-    if (!tmap_mnmajor(&tx, X, K, T) || !tmap_mnmajor(&tv, sV, r, T)) return QLORA_ERR_CUDA;
+    if (!tmap_mnmajor(&tx, X, K, T) || !tmap_mnmajor(&tv, sV, r, T)) return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
     if (int e = launch_skinny_bn<Skinny::kGrad>(bn, tx, tv, K, T, part, cdiv(K, 128) * 128 * bn, st)) return e;
     if (int e = reduce_after(part, K, T, r, bn, 1.0f, dA, Red::kTransF32, st)) return e;
   }
   {
     // dB[n][j] = sum_t dY[t][n] sU[t][j]
     CUtensorMap tdy, tu;
-    if (!tmap_mnmajor(&tdy, dY, N, T) || !tmap_mnmajor(&tu, sU, r, T)) return QLORA_ERR_CUDA;
+    if (!tmap_mnmajor(&tdy, dY, N, T) || !tmap_mnmajor(&tu, sU, r, T)) return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
     if (int e = launch_skinny_bn<Skinny::kGrad>(bn, tdy, tu, N, T, part, cdiv(N, 128) * 128 * bn, st)) return e;
     if (int e = reduce_after(part, N, T, r, bn, 1.0f, dB, Red::kRowsF32, st)) return e;
   }
@@ -800,11 +826,11 @@ int qlora_linear_bwd(const void* dY, const void* X, int64_t T, const qlora_nf4_t
 
 int qlora_get_status(int* device_status, qlora_stream_t stream) {
   if (!device_status) return QLORA_ERR_INVALID_ARG;
-  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
   unsigned v = 0, zero = 0;
   if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess ||
       cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess)
-    return QLORA_ERR_CUDA;
+    return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
   *device_status = static_cast<int>(v);
   if (v & kStatusTimeout) return QLORA_ERR_TIMEOUT;
   if (v & kStatusNonfinite) return QLORA_ERR_NONFINITE;
