@@ -15,6 +15,9 @@ What it computes, in the pages' order (citations are to the source pages by titl
                quantization of the block constants, and dequantization
                [PEFT page, "Block-wise quantization in one page", "Double quantization",
                 "The real way"]
+  codebook_study.py  the codebook comparison: any sorted codebook of up to 16 levels with fp32 block
+               constants, code entropy and RMS error, and Lloyd's algorithm
+               [PEFT page, "NF4, derived from normal quantiles"]
   linear.py    the QLoRA linear layer, forward and backward, in fp64
                [QLoRA explainer, prism.theerrors.in, "Putting it together";
                 PEFT page, "Paged optimizers, and QLoRA end to end"]
@@ -31,5 +34,6 @@ from .codec import (BLOCK, DQ_BLOCK, num_blocks, num_groups, storage_bytes, absm
                     double_quantize, double_dequantize, quantize, dequantize, NF4Tensor,
                     quantize_single, dequantize_single, storage_bytes_single, NF4SingleTensor)
 from .linear import linear_fwd, linear_bwd
+from . import codebook_study
 
 __all__ = [n for n in dir() if not n.startswith("_")]
