@@ -575,6 +575,79 @@ def run_codec_sweep(args):
     return 0
 
 
+STUDY_SHAPE = (8192, 8192)
+STUDY_LLOYD_STEPS = 30
+
+
+def run_codebook_study(args):
+    """The page's codebook comparison at scale through the library's kernels: an 8192 x 8192 Gaussian
+    matrix (2^26 elements, 256 MB fp32, larger than L2) in blocks of 64 with fp32 constants, under
+    symmetric int4, the {-8..7}/8 grid, NF4 and Lloyd's codebook (30 device steps from NF4)."""
+    import numpy as np
+    import torch
+    import synth
+    import bit_nf4_quantized_14_b200 as q
+    peaks, kind = load_peaks()
+    device = torch.device("cuda", 0)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    x = torch.from_numpy(synth.normal_f32(STUDY_SHAPE, 1.0, 0, 17).reshape(-1)).to(device)
+    n = x.numel()
+    nf4, _ = q.codebook()
+    codes = torch.empty(-(-n // 2), dtype=torch.uint8, device=device)
+    absmax = torch.empty(-(-n // 64), dtype=torch.float32, device=device)
+    out32 = torch.empty(n, dtype=torch.float32, device=device)
+    st = torch.empty(q.CODEBOOK_STATS_LEN, dtype=torch.float64, device=device)
+    ws = torch.empty(q.codebook_stats_workspace_bytes(n), dtype=torch.uint8, device=device)
+    stored = 0.5 + 4 / 64
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record()
+    lloyd_lv, hist = q.lloyd(x, nf4, STUDY_LLOYD_STEPS)
+    t1.record()
+    torch.cuda.synchronize()
+    lloyd_ms = t0.elapsed_time(t1) / (STUDY_LLOYD_STEPS + 1)
+    books = {"int4_symmetric": np.arange(-7, 8, dtype=np.float32) / np.float32(7),
+             "grid_16": np.arange(-8, 8, dtype=np.float32) / np.float32(8), "nf4": nf4, "lloyd": lloyd_lv}
+    cases = {}
+    for name, lv in books.items():
+        row = {"levels": [float(v) for v in lv]}
+        for label, fn, bpe in (
+                ("quantize", lambda: q.codebook_quantize(x, lv, codes, absmax), 4 + stored),
+                ("dequantize_fp32", lambda: q.codebook_dequantize(codes, absmax, n, lv, torch.float32, out32), stored + 4),
+                ("stats", lambda: q.codebook_stats(x, codes, absmax, lv, st, ws), 4 + stored)):
+            ms = time_calls(fn, flush, args.steps, args.warmup)
+            row[label] = {"us": round(ms * 1e3, 2), "GB/s": round(n * bpe / (ms / 1e3) / 1e9, 1),
+                          "frac": round(n * bpe / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
+        q.codebook_quantize(x, lv, codes, absmax)
+        d = q.stats_dict(q.codebook_stats(x, codes, absmax, lv, st, ws), lv.size)
+        row.update(entropy_bits=round(d["entropy_bits"], 4), rms=d["rms"])
+        cases[name] = row
+    figures = {
+        "entropy_bits_nf4": cases["nf4"]["entropy_bits"],
+        "entropy_bits_int4_symmetric": cases["int4_symmetric"]["entropy_bits"],
+        "rms_reduction_nf4_vs_int4": round(1 - cases["nf4"]["rms"] / cases["int4_symmetric"]["rms"], 4),
+        "lloyd_gain_over_nf4": round(1 - cases["lloyd"]["rms"] / cases["nf4"]["rms"], 4),
+        "page": {"entropy_bits_nf4": 3.88, "entropy_bits_int4_symmetric": 3.50, "rms_reduction_nf4_vs_int4": 0.15,
+                 "lloyd_gain_over_nf4": 0.05}}
+    status = q.get_status()
+    print(json.dumps({"metric": "Lloyd step (codebook quantize + statistics) throughput on the codebook "
+                                "comparison matrix",
+                      "value": round(n / (lloyd_ms / 1e3) / 1e9, 2), "unit": "G elements/s", "n_gpus": 1,
+                      "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+                      "ms_per_lloyd_step": round(lloyd_ms, 4), "dtype": "f32 in, u8 codes + fp32 constants, f64 sums",
+                      "data": "synthetic",
+                      "config": {"workload": "8192 x 8192 N(0, 1) fp32 matrix (2^26 elements), blocks of 64, fp32 "
+                                             "constants; codebooks int4 {-7..7}/7, grid {-8..7}/8, NF4, Lloyd "
+                                             f"({STUDY_LLOYD_STEPS} device steps from NF4)",
+                                 "l2": "flushed (512 MB write) before every timed codec call; the Lloyd loop runs "
+                                       "back to back (input 256 MB > L2)"},
+                      "roofline": {"bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                                   "peak_source": f"{kind} (HBM copy)"},
+                      "figures": figures, "rms_history": hist, "cases": cases, "device_status": status}), flush=True)
+    return 0
+
+
 LLAMA65B_LAYERS, LLAMA65B_TOKENS = 80, 512
 LLAMA65B_WORKLOAD = ("LLaMA-65B-shaped decoder linears: 80 layers x (q, k, v, o 8192x8192; gate, up 22016x8192; "
                      "down 8192x22016) as NF4 + LoRA r = 64, alpha = 16; one step = the 560 linear forward + "
@@ -789,7 +862,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) measurement")
     ap.add_argument("--workload", choices=["llama7b_step", "decode", "codec_sweep", "llama65b_linears",
-                                           "llama65b_train"],
+                                           "llama65b_train", "codebook_study"],
                     default="llama7b_step",
                     help="llama7b_step (the headline line), or the decode / codec-sweep / 65B-step measurement lines")
     ap.add_argument("--shapes", default="all",
@@ -810,6 +883,8 @@ def main(argv=None):
         return run_llama65b(args)
     if args.workload == "llama65b_train":
         return run_llama65b_train(args)
+    if args.workload == "codebook_study":
+        return run_codebook_study(args)
     return run_gpu(args)
 
 

@@ -8,6 +8,7 @@ include/qlora_nf4.h:
     dequantize(q, dtype)             -> tensor        (qlora_nf4_dequantize)
     linear_fwd(X, q, A, B, alpha)    -> (Y, U)        (qlora_linear_fwd)
     linear_bwd(dY, X, q, A, B, alpha, U) -> (dX, dA, dB)   (qlora_linear_bwd)
+    codebook_quantize / codebook_dequantize / codebook_stats   (qlora_codebook_*)
 
 The shared library is loaded on first use (so that the build step, a submodule of this package, can run
 before it exists); a call made while it is not built raises ImportError. There is no fallback
@@ -68,6 +69,10 @@ def _open() -> ctypes.CDLL:
         "qlora_nf4_dequantize": [P(_NF4Struct), vp, i32, vp],
         "qlora_nf4_quantize_single": [vp, i32, i64, i64, vp, vp, vp],
         "qlora_nf4_dequantize_single": [vp, vp, i64, i64, vp, i32, vp],
+        "qlora_codebook_quantize": [vp, i32, i64, P(ctypes.c_float), i32, vp, vp, vp],
+        "qlora_codebook_dequantize": [vp, vp, i64, P(ctypes.c_float), i32, vp, i32, vp],
+        "qlora_codebook_stats_workspace": [i64, P(sz)],
+        "qlora_codebook_stats": [vp, i32, vp, vp, i64, P(ctypes.c_float), i32, vp, vp, sz, vp],
         "qlora_linear_workspace": [i64, i64, i64, i32, P(sz)],
         "qlora_linear_fwd": [vp, i64, P(_NF4Struct), vp, vp, i32, ctypes.c_float, vp, vp, vp, sz, vp],
         "qlora_linear_bwd": [vp, vp, i64, P(_NF4Struct), vp, vp, i32, ctypes.c_float, vp, vp, vp, vp,
@@ -221,6 +226,94 @@ def dequantize_single(q: NF4SingleWeight, dtype=torch.bfloat16, out: torch.Tenso
                                               QLORA_F32 if dtype == torch.float32 else QLORA_BF16, _stream(stream)),
            "qlora_nf4_dequantize_single")
     return o
+
+
+# ---- codebook comparison: any sorted codebook of 2..16 levels, fp32 block constants -------------------
+
+CODEBOOK_STATS_LEN = 51
+
+
+def _levels(levels):
+    lv = np.ascontiguousarray(np.asarray(levels, dtype=np.float32).reshape(-1))
+    return (ctypes.c_float * lv.size)(*lv.tolist()), int(lv.size)
+
+
+def codebook_quantize(w: torch.Tensor, levels, codes: torch.Tensor | None = None,
+                      absmax: torch.Tensor | None = None, stream=None):
+    """(codes uint8[ceil(n/2)], absmax float32[ceil(n/64)]) of a contiguous CUDA fp32/bf16 tensor under
+    `levels` (qlora_codebook_quantize)."""
+    if w.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("codebook_quantize: w must be float32 or bfloat16")
+    _need(w, w.dtype, "w")
+    n = w.numel()
+    c = codes if codes is not None else torch.empty(-(-n // 2), dtype=torch.uint8, device=w.device)
+    a = absmax if absmax is not None else torch.empty(-(-n // 64), dtype=torch.float32, device=w.device)
+    lv, nl = _levels(levels)
+    _check(load().qlora_codebook_quantize(_ptr(w), QLORA_F32 if w.dtype == torch.float32 else QLORA_BF16, n, lv, nl,
+                                          _ptr(c), _ptr(a), _stream(stream)), "qlora_codebook_quantize")
+    return c, a
+
+
+def codebook_dequantize(codes: torch.Tensor, absmax: torch.Tensor, n: int, levels, dtype=torch.float32,
+                        out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    if dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("codebook_dequantize: dtype must be float32 or bfloat16")
+    o = out if out is not None else torch.empty(n, dtype=dtype, device=codes.device)
+    _need(o, dtype, "out")
+    lv, nl = _levels(levels)
+    _check(load().qlora_codebook_dequantize(_ptr(codes), _ptr(absmax), n, lv, nl, _ptr(o),
+                                            QLORA_F32 if dtype == torch.float32 else QLORA_BF16, _stream(stream)),
+           "qlora_codebook_dequantize")
+    return o
+
+
+def codebook_stats_workspace_bytes(n: int) -> int:
+    b = ctypes.c_size_t()
+    _check(load().qlora_codebook_stats_workspace(n, ctypes.byref(b)), "qlora_codebook_stats_workspace")
+    return b.value
+
+
+def codebook_stats(w: torch.Tensor, codes: torch.Tensor, absmax: torch.Tensor, levels,
+                   out: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The CODEBOOK_STATS_LEN float64 values of qlora_codebook_stats, on the device."""
+    _need(w, w.dtype, "w")
+    n = w.numel()
+    o = out if out is not None else torch.empty(CODEBOOK_STATS_LEN, dtype=torch.float64, device=w.device)
+    _need(o, torch.float64, "out")
+    ws = workspace if workspace is not None else torch.empty(codebook_stats_workspace_bytes(n), dtype=torch.uint8,
+                                                             device=w.device)
+    lv, nl = _levels(levels)
+    _check(load().qlora_codebook_stats(_ptr(w), QLORA_F32 if w.dtype == torch.float32 else QLORA_BF16, _ptr(codes),
+                                       _ptr(absmax), n, lv, nl, _ptr(o), _ptr(ws), ws.numel(), _stream(stream)),
+           "qlora_codebook_stats")
+    return o
+
+
+def stats_dict(stats: torch.Tensor, nlevels: int) -> dict:
+    """The fields of a qlora_codebook_stats result, copied to the host."""
+    v = stats.detach().cpu().numpy()
+    return {"counts": v[0:16].astype(np.int64), "sums": v[16:32].copy(), "sse": float(v[32]),
+            "entropy_bits": float(v[33]), "rms": float(v[34]), "centroids": v[35:35 + nlevels].astype(np.float32)}
+
+
+def lloyd(w: torch.Tensor, levels, iters: int, stream=None):
+    """Lloyd's algorithm on the device: `iters` rounds of codebook_quantize + codebook_stats, each taking
+    the kernel's updated levels. Returns the final levels (numpy fp32) and the RMS error before each step
+    and after the last."""
+    lv = np.asarray(levels, dtype=np.float32).copy()
+    n = w.numel()
+    codes = torch.empty(-(-n // 2), dtype=torch.uint8, device=w.device)
+    absmax = torch.empty(-(-n // 64), dtype=torch.float32, device=w.device)
+    ws = torch.empty(codebook_stats_workspace_bytes(n), dtype=torch.uint8, device=w.device)
+    st = torch.empty(CODEBOOK_STATS_LEN, dtype=torch.float64, device=w.device)
+    hist = []
+    for k in range(iters + 1):
+        codebook_quantize(w, lv, codes, absmax, stream)
+        d = stats_dict(codebook_stats(w, codes, absmax, lv, st, ws, stream), lv.size)
+        hist.append(d["rms"])
+        if k < iters:
+            lv = d["centroids"]
+    return lv, hist
 
 
 NOALLOC_MAX_NUMEL = 1 << 26

@@ -5,6 +5,8 @@
 
 #include <algorithm>
 #include <climits>
+#include <cmath>
+#include <limits>
 #include <cstdio>
 #include <cstdlib>
 #include <atomic>
@@ -54,31 +56,56 @@ const CodebookArg& codebook() {
   return cb;
 }
 
-// The quantizer's bucket table: bucket b (1..31) covers t = w/a in [(b - 16.5)/15, (b - 15.5)/15],
-// widened by kBucketWiden for the approximate reciprocal; lo(b) counts the thresholds below it. Valid
-// only if every widened bucket holds at most one threshold (true for the NF4 thresholds, whose closest
-// pair is 0.0805 apart against a bucket width of 0.0667); checked here once.
+// The quantizer's bucket table for a codebook of nl levels: bucket b (1..31) covers t = w/a in
+// [(b - 16.5)/15, (b - 15.5)/15], widened by kBucketWiden for the approximate reciprocal; lo(b) counts the
+// thresholds below it. Valid only if every widened bucket holds at most one threshold (true for the NF4
+// thresholds, whose closest pair is 0.0805 apart against a bucket width of 0.0667). Also sets the code of
+// an all-zero block: the level of least magnitude, the lower index on a tie (NF4: 7, its exact zero).
+bool build_buckets(const CodebookArg& cb, int nl, BucketArg* out) {
+  *out = BucketArg{};
+  bool ok = true;
+  for (int b = 0; b < 32; ++b) {
+    const double jl = (b - 16.5) / 15.0 - kBucketWiden, ju = (b - 15.5) / 15.0 + kBucketWiden;
+    int lo = 0, inside = 0;
+    for (int j = 0; j < nl - 1; ++j) {
+      const double t = cb.thresholds[j];
+      lo += (t < jl) ? 1 : 0;
+      inside += (t >= jl && t <= ju) ? 1 : 0;
+    }
+    if (inside > 1) ok = false;
+    out->lo_nibbles[b / 8] |= static_cast<uint32_t>(lo) << (4 * (b % 8));
+  }
+  int z = 0;
+  for (int j = 1; j < nl; ++j)
+    if (std::fabs(cb.levels[j]) < std::fabs(cb.levels[z])) z = j;
+  out->zero_codes = 0x11111111u * static_cast<uint32_t>(z);
+  return ok;
+}
+
 struct Buckets { BucketArg arg; bool ok; };
 const Buckets& buckets() {
   static Buckets bk;
   static std::once_flag once;
-  std::call_once(once, [] {
-    const CodebookArg& cb = codebook();
-    bk.arg = BucketArg{};
-    bk.ok = true;
-    for (int b = 0; b < 32; ++b) {
-      const double jl = (b - 16.5) / 15.0 - kBucketWiden, ju = (b - 15.5) / 15.0 + kBucketWiden;
-      int lo = 0, inside = 0;
-      for (int j = 0; j < 15; ++j) {
-        const double t = cb.thresholds[j];
-        lo += (t < jl) ? 1 : 0;
-        inside += (t >= jl && t <= ju) ? 1 : 0;
-      }
-      if (inside > 1) bk.ok = false;
-      bk.arg.lo_nibbles[b / 8] |= static_cast<uint32_t>(lo) << (4 * (b % 8));
-    }
-  });
+  std::call_once(once, [] { bk.ok = build_buckets(codebook(), 16, &bk.arg); });
   return bk;
+}
+
+// Kernel arguments for a caller's codebook (host array of nl levels): false unless 2 <= nl <= 16, the
+// levels are finite, in [-1, 1] and strictly ascending, and the bucket table is valid. Thresholds are the
+// fp32 roundings of the fp64 level midpoints; thresholds past nl - 1 are +inf (never crossed) and levels
+// past nl are 0 (never looked up).
+bool make_codebook(const float* lv, int nl, CodebookArg* cb, BucketArg* bk) {
+  if (!lv || nl < 2 || nl > 16) return false;
+  for (int j = 0; j < nl; ++j) {
+    if (!(std::fabs(lv[j]) <= 1.0f)) return false;             // also rejects NaN
+    if (j > 0 && !(lv[j] > lv[j - 1])) return false;
+  }
+  *cb = CodebookArg{};
+  for (int j = 0; j < 16; ++j) cb->levels[j] = j < nl ? lv[j] : 0.0f;
+  for (int j = 0; j < 15; ++j)
+    cb->thresholds[j] = j < nl - 1 ? static_cast<float>((static_cast<double>(lv[j]) + lv[j + 1]) / 2.0)
+                                   : std::numeric_limits<float>::infinity();
+  return build_buckets(*cb, nl, bk);
 }
 
 // Launch with programmatic stream serialization: the kernel may start while its predecessor in the
@@ -600,7 +627,8 @@ int run_quantize(const void* w, int w_dtype, int64_t n, const qlora_nf4_tensor* 
 
 // The bulk-copy dequantizer in either constant format (double-quantized, or fp32 per block).
 int launch_dequant(bool bf16, bool single, const uint8_t* codes, const uint8_t* e4m3, const float* s2,
-                   const float* mu, const float* c1, int64_t n, void* out, int sms, cudaStream_t st) {
+                   const float* mu, const float* c1, int64_t n, void* out, int sms, cudaStream_t st,
+                   const CodebookArg& cb) {
   auto kern = bf16 ? (single ? nf4_dequantize_kernel<true, true> : nf4_dequantize_kernel<true, false>)
                    : (single ? nf4_dequantize_kernel<false, true> : nf4_dequantize_kernel<false, false>);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDeqSmemBytes) != cudaSuccess)
@@ -610,9 +638,27 @@ int launch_dequant(bool bf16, bool single, const uint8_t* codes, const uint8_t* 
     return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
   const unsigned grid = static_cast<unsigned>(
       std::max<int64_t>(1, std::min<int64_t>(cdiv(n, kGroupElems), int64_t(sms) * std::max(per_sm, 1))));
-  kern<<<grid, kDeqThreads, kDeqSmemBytes, st>>>(codes, e4m3, s2, mu, c1, n, out, codebook());
+  kern<<<grid, kDeqThreads, kDeqSmemBytes, st>>>(codes, e4m3, s2, mu, c1, n, out, cb);
   return launched();
 }
+
+// Pass 1 alone, with fp32 block constants kept as they are (no slab sums, no mean pass).
+int launch_pass1_single(const void* w, int w_dtype, int64_t n, uint8_t* codes, float* absmax,
+                        const CodebookArg& cb, const BucketArg& bk, int sms, cudaStream_t st) {
+  const int64_t ns = cdiv(n, kSlabElems);
+  const unsigned g1 =
+      static_cast<unsigned>(std::min<int64_t>(cdiv(ns, kQuantThreads / 32), int64_t(sms) * kQuantMinBlocks));
+  if (w_dtype == QLORA_F32)
+    nf4_quantize_pass1<float><<<g1, kQuantThreads, 0, st>>>(static_cast<const float*>(w), n, codes, absmax,
+                                                             nullptr, ns, cb, bk, nullptr);
+  else
+    nf4_quantize_pass1<__nv_bfloat16><<<g1, kQuantThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(w), n, codes,
+                                                                     absmax, nullptr, ns, cb, bk, nullptr);
+  return launched();
+}
+
+static_assert(kStatOut == QLORA_CODEBOOK_STATS_LEN, "codebook statistics layout");
+int64_t stat_ctas(int64_t n) { return std::min<int64_t>(cdiv(cdiv(n, kStepElems), kStatThreads / 32), kStatMaxCtas); }
 }  // namespace
 }  // namespace qnf4
 
@@ -687,7 +733,7 @@ int qlora_nf4_dequantize(const qlora_nf4_tensor* q, void* out, int out_dtype, ql
   const int64_t n = q->rows * q->cols;
   ProfScope prof(QLORA_PROF_DEQUANTIZE, st);
   return launch_dequant(out_dtype == QLORA_BF16, false, q->codes, q->absmax_e4m3, q->scale2, q->offset, nullptr, n,
-                        out, sms, st);
+                        out, sms, st, codebook());
 }
 
 int qlora_nf4_quantize_single(const void* w, int w_dtype, int64_t rows, int64_t cols, void* codes, float* absmax,
@@ -701,17 +747,9 @@ int qlora_nf4_quantize_single(const void* w, int w_dtype, int64_t rows, int64_t 
   const Buckets& bk = buckets();
   if (!bk.ok) return QLORA_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t n = rows * cols, ns = cdiv(n, kSlabElems);
-  const unsigned g1 = static_cast<unsigned>(std::min<int64_t>(cdiv(ns, kQuantThreads / 32), int64_t(sms) * kQuantMinBlocks));
   ProfScope prof(QLORA_PROF_QUANTIZE, st);
-  uint8_t* c = static_cast<uint8_t*>(codes);
-  if (w_dtype == QLORA_F32)
-    nf4_quantize_pass1<float><<<g1, kQuantThreads, 0, st>>>(static_cast<const float*>(w), n, c, absmax, nullptr, ns,
-                                                             codebook(), bk.arg, nullptr);
-  else
-    nf4_quantize_pass1<__nv_bfloat16><<<g1, kQuantThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(w), n, c,
-                                                                     absmax, nullptr, ns, codebook(), bk.arg, nullptr);
-  return launched();
+  return launch_pass1_single(w, w_dtype, rows * cols, static_cast<uint8_t*>(codes), absmax, codebook(), bk.arg, sms,
+                             st);
 }
 
 int qlora_nf4_dequantize_single(const void* codes, const float* absmax, int64_t rows, int64_t cols, void* out,
@@ -725,7 +763,75 @@ int qlora_nf4_dequantize_single(const void* codes, const float* absmax, int64_t 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   ProfScope prof(QLORA_PROF_DEQUANTIZE, st);
   return launch_dequant(out_dtype == QLORA_BF16, true, static_cast<const uint8_t*>(codes), nullptr, nullptr, nullptr,
-                        absmax, rows * cols, out, sms, st);
+                        absmax, rows * cols, out, sms, st, codebook());
+}
+
+int qlora_codebook_quantize(const void* w, int w_dtype, int64_t n, const float* levels, int nlevels, void* codes,
+                            float* absmax, qlora_stream_t stream) {
+  if (!w || !codes || !absmax) return QLORA_ERR_INVALID_ARG;
+  if (w_dtype != QLORA_F32 && w_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
+  if (n <= 0 || n > kMaxNumel) return QLORA_ERR_SHAPE;
+  CodebookArg cb;
+  BucketArg bk;
+  if (!make_codebook(levels, nlevels, &cb, &bk)) return QLORA_ERR_CODEBOOK;
+  if (!aligned16(w) || !aligned16(codes) || !aligned16(absmax)) return QLORA_ERR_ALIGNMENT;
+  int sms = 0;
+  if (int e = check_device(&sms)) return e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  ProfScope prof(QLORA_PROF_QUANTIZE, st);
+  return launch_pass1_single(w, w_dtype, n, static_cast<uint8_t*>(codes), absmax, cb, bk, sms, st);
+}
+
+int qlora_codebook_dequantize(const void* codes, const float* absmax, int64_t n, const float* levels, int nlevels,
+                              void* out, int out_dtype, qlora_stream_t stream) {
+  if (!codes || !absmax || !out) return QLORA_ERR_INVALID_ARG;
+  if (out_dtype != QLORA_F32 && out_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
+  if (n <= 0 || n > kMaxNumel) return QLORA_ERR_SHAPE;
+  CodebookArg cb;
+  BucketArg bk;
+  if (!make_codebook(levels, nlevels, &cb, &bk)) return QLORA_ERR_CODEBOOK;
+  if (!aligned16(codes) || !aligned16(absmax) || !aligned16(out)) return QLORA_ERR_ALIGNMENT;
+  int sms = 0;
+  if (int e = check_device(&sms)) return e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  ProfScope prof(QLORA_PROF_DEQUANTIZE, st);
+  return launch_dequant(out_dtype == QLORA_BF16, true, static_cast<const uint8_t*>(codes), nullptr, nullptr, nullptr,
+                        absmax, n, out, sms, st, cb);
+}
+
+int qlora_codebook_stats_workspace(int64_t n, size_t* bytes) {
+  if (!bytes) return QLORA_ERR_INVALID_ARG;
+  if (n <= 0 || n > kMaxNumel) return QLORA_ERR_SHAPE;
+  *bytes = align256(static_cast<size_t>(stat_ctas(n)) * kStatVals * sizeof(double));
+  return QLORA_OK;
+}
+
+int qlora_codebook_stats(const void* w, int w_dtype, const void* codes, const float* absmax, int64_t n,
+                         const float* levels, int nlevels, double* stats, void* workspace, size_t workspace_bytes,
+                         qlora_stream_t stream) {
+  if (!w || !codes || !absmax || !stats) return QLORA_ERR_INVALID_ARG;
+  if (w_dtype != QLORA_F32 && w_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
+  if (n <= 0 || n > kMaxNumel) return QLORA_ERR_SHAPE;
+  CodebookArg cb;
+  BucketArg bk;
+  if (!make_codebook(levels, nlevels, &cb, &bk)) return QLORA_ERR_CODEBOOK;
+  const int64_t G = stat_ctas(n);
+  if (!workspace || workspace_bytes < static_cast<size_t>(G) * kStatVals * sizeof(double)) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(w) || !aligned16(codes) || !aligned16(absmax) || !aligned16(stats) || !aligned16(workspace))
+    return QLORA_ERR_ALIGNMENT;
+  if (int e = check_device(nullptr)) return e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  double* part = static_cast<double*>(workspace);
+  const uint8_t* c = static_cast<const uint8_t*>(codes);
+  if (w_dtype == QLORA_F32)
+    codebook_stats_partial<float><<<static_cast<unsigned>(G), kStatThreads, 0, st>>>(static_cast<const float*>(w), c,
+                                                                                    absmax, n, cb, part);
+  else
+    codebook_stats_partial<__nv_bfloat16><<<static_cast<unsigned>(G), kStatThreads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(w), c, absmax, n, cb, part);
+  if (int e = launched()) return e;
+  codebook_stats_final<<<1, 64, 0, st>>>(part, static_cast<int>(G), n, cb, nlevels, stats);
+  return launched();
 }
 
 int qlora_linear_workspace(int64_t T, int64_t N, int64_t K, int r, size_t* bytes) {
@@ -849,6 +955,7 @@ const char* qlora_error_string(int code) {
     case QLORA_ERR_TIMEOUT: return "a kernel gave up waiting (bounded wait expired)";
     case QLORA_ERR_UNSUPPORTED: return "device is not an sm_100 GPU";
     case QLORA_ERR_TOO_LARGE: return "input exceeds the fixed scratch of the no-allocation quantize (2^26 elements)";
+    case QLORA_ERR_CODEBOOK: return "codebook not 2..16 ascending levels in [-1, 1], or two thresholds within one bucket";
   }
   return "unknown error code";
 }

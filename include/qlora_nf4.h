@@ -49,7 +49,8 @@ enum qlora_status_code {
   QLORA_ERR_NONFINITE = -6,    /* (status) a quantized input held Inf or NaN                        */
   QLORA_ERR_TIMEOUT = -7,      /* (status) a kernel's bounded wait gave up; its outputs are invalid */
   QLORA_ERR_UNSUPPORTED = -8,  /* the current device is not an sm_100 (B200-class) GPU             */
-  QLORA_ERR_TOO_LARGE = -9     /* input larger than the fixed scratch of qlora_nf4_quantize_noalloc */
+  QLORA_ERR_TOO_LARGE = -9,    /* input larger than the fixed scratch of qlora_nf4_quantize_noalloc */
+  QLORA_ERR_CODEBOOK = -10     /* codebook not 2..16 ascending levels in [-1, 1], or too dense      */
 };
 
 /* Bits of the device status word (qlora_get_status). */
@@ -166,6 +167,48 @@ int qlora_nf4_quantize_single(const void* w, int w_dtype, int64_t rows, int64_t 
                               float* absmax, qlora_stream_t stream);
 int qlora_nf4_dequantize_single(const void* codes, const float* absmax, int64_t rows, int64_t cols,
                                 void* out, int out_dtype, qlora_stream_t stream);
+
+/*
+ * Codebook comparison [PEFT "NF4, derived from normal quantiles": a Gaussian matrix quantized in blocks
+ * of 64 with the symmetric int4 grid {-7..7}/7, the grid {-8..7}/8, NF4 and Lloyd's least-squares
+ * codebook, compared by code entropy and RMS error; "Block-wise quantization in one page"]. The same
+ * quantizer and dequantizer as the NF4 calls, with fp32 block constants and the caller's codebook.
+ *
+ * levels (host, nlevels fp32 values): 2 <= nlevels <= 16, strictly ascending, every |level| <= 1.
+ * Thresholds are T_j = fp32((level_j + level_{j+1}) / 2), the sum formed in fp64; the code of w in a
+ * block with absmax a > 0 is #{j : w > T_j * a} evaluated exactly (at most nlevels - 1), and an all-zero
+ * block codes as the index of the level of least magnitude (the lower one on a tie). The quantizer looks
+ * thresholds up by buckets of width 1/15 in w / a, so every bucket (widened by 2^-18) may hold at most
+ * one threshold: any two thresholds more than 1/15 + 2^-17 apart always pass (the NF4, int4, {-8..7}/8
+ * and Lloyd codebooks do). A codebook that breaks a rule returns QLORA_ERR_CODEBOOK, before any device
+ * call. n is the element count of a dense tensor (1 <= n <= 2^40); the caller allocates `codes`
+ * (ceil(n/2) bytes, two codes per byte, even element in the high nibble) and `absmax` (ceil(n/64) fp32).
+ *   qlora_codebook_quantize    w (QLORA_F32 or QLORA_BF16) -> codes, absmax. A non-finite input sets
+ *                              QLORA_STATUS_NONFINITE. With the NF4 levels the output equals
+ *                              qlora_nf4_quantize_single's.
+ *   qlora_codebook_dequantize  w_hat = fp32(level[code] * absmax[block]), bf16 (RNE) for QLORA_BF16.
+ *   qlora_codebook_stats       what the codebook did to w (w, codes and absmax as written by
+ *                              qlora_codebook_quantize with the same levels; w finite). `stats` is a
+ *                              device array of QLORA_CODEBOOK_STATS_LEN doubles:
+ *       [0..15]   count_j, the number of elements with code j
+ *       [16..31]  sum_j, the sum of u = w / a (fp64, correctly rounded; 0 in an all-zero block) over them
+ *       [32]      sum over all elements of (w_hat - w)^2 in fp64, w_hat as qlora_codebook_dequantize's fp32
+ *       [33]      code entropy in bits, -sum_j p_j log2 p_j with p_j = count_j / n
+ *       [34]      RMS error, sqrt([32] / n)
+ *       [35..50]  one step of Lloyd's algorithm: fp32(sum_j / count_j), or level_j where count_j = 0
+ *                 (entries past nlevels hold 0)
+ *     Sums run in a fixed order for a given n and device, so the result is deterministic.
+ *     `workspace` >= qlora_codebook_stats_workspace(n) bytes (device).
+ */
+#define QLORA_CODEBOOK_STATS_LEN 51
+int qlora_codebook_quantize(const void* w, int w_dtype, int64_t n, const float* levels, int nlevels,
+                            void* codes, float* absmax, qlora_stream_t stream);
+int qlora_codebook_dequantize(const void* codes, const float* absmax, int64_t n, const float* levels,
+                              int nlevels, void* out, int out_dtype, qlora_stream_t stream);
+int qlora_codebook_stats_workspace(int64_t n, size_t* bytes);
+int qlora_codebook_stats(const void* w, int w_dtype, const void* codes, const float* absmax, int64_t n,
+                         const float* levels, int nlevels, double* stats, void* workspace,
+                         size_t workspace_bytes, qlora_stream_t stream);
 
 /*
  * Device workspace bytes for qlora_linear_fwd / qlora_linear_bwd with T tokens, weight N x K (out x in)

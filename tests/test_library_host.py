@@ -124,3 +124,31 @@ def test_error_strings(q):
     for c in range(-9, 1):
         assert len(q.lib.qlora_error_string(c)) > 0
     assert q.lib.qlora_error_string(-99) == b"unknown error code"
+
+
+def test_codebook_calls_reject_bad_codebooks_before_any_cuda_call(q):
+    """Unsorted, out-of-range, non-finite, too few or too many levels, and two thresholds closer than
+    one bucket (1/15 in w / a) all return QLORA_ERR_CODEBOOK; the oracle rejects the same level lists."""
+    from oracle import codebook_study as CS
+    L = q.lib
+    F = ctypes.c_float
+    W, C, A, OUT, WS = V(0x300000), V(0x310000), V(0x320000), V(0x330000), V(0x340000)
+    bad = [[0.5], [0.0, 0.0], [0.5, -0.5], [-1.0, 1.5], [-1.0, float("nan")], list(np.linspace(-1, 1, 17))]
+    dense = [-1.0, -0.02, 0.0, 0.02, 1.0]            # midpoints -0.01 and 0.01 share a bucket
+    for lv in bad + [dense]:
+        arr = (F * len(lv))(*lv)
+        assert L.qlora_codebook_quantize(W, 0, 4096, arr, len(lv), C, A, None) == -10, lv
+        assert L.qlora_codebook_dequantize(C, A, 4096, arr, len(lv), OUT, 1, None) == -10, lv
+        assert L.qlora_codebook_stats(W, 0, C, A, 4096, arr, len(lv), OUT, WS, 1 << 20, None) == -10, lv
+        if lv is not dense:
+            with pytest.raises(ValueError):
+                CS.check_levels(lv)
+    good = (F * 15)(*(np.arange(-7, 8, dtype=np.float32) / np.float32(7)).tolist())
+    assert L.qlora_codebook_quantize(W, 0, 0, good, 15, C, A, None) == -2
+    assert L.qlora_codebook_quantize(W, 5, 64, good, 15, C, A, None) == -1
+    assert L.qlora_codebook_quantize(V(0x300004), 0, 64, good, 15, C, A, None) == -3
+    assert L.qlora_codebook_stats(W, 0, C, A, 64, good, 15, OUT, WS, 0, None) == -4
+    assert L.qlora_codebook_stats(W, 0, C, A, 64, good, 15, OUT, None, 1 << 20, None) == -4
+    b = ctypes.c_size_t()
+    assert L.qlora_codebook_stats_workspace(1 << 30, ctypes.byref(b)) == 0 and b.value >= 33 * 8
+    assert L.qlora_codebook_stats_workspace(0, ctypes.byref(b)) == -2
