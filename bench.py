@@ -26,6 +26,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import sys
 import time
@@ -193,25 +194,97 @@ def torch_bf16():
     return torch.bfloat16
 
 
-def source_hash():
+# The headers each timed kernel class is compiled from (tile shapes, stage counts and CTA shapes are fixed
+# there; the host sizes the persistent grids from the SM count alone); a DRAM-traffic record taken with ncu
+# is used only while these files are unchanged.
+KERNEL_SOURCES = {
+    "fwd_gemm": ("common.cuh", "codec.cuh", "gemm_nf4w.cuh"),
+    "bwd_gemm": ("common.cuh", "codec.cuh", "gemm_nf4w.cuh"),
+    "quantize": ("common.cuh", "codec.cuh"),
+    "dequantize": ("common.cuh", "codec.cuh"),
+}
+
+
+def source_hash(cls: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_nf4_quantized_14_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in KERNEL_SOURCES[cls]:
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def traffic_for(cls: str):
     """DRAM bytes per launch of a kernel class from the committed ncu summary, if it was taken on the
-    current kernel sources."""
+    class's current sources."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
     e = d.get(cls)
-    if not e or e.get("source_hash") != source_hash():
+    if not e or e.get("source_hash") != source_hash(cls):
         return None
     return e.get("bytes_per_launch")
+
+
+def kernel_class(name: str):
+    """(profiling class, label) of a kernel name as ncu prints it; the class is the library's timing class
+    whose interval holds the launch (None for kernels outside the four measured classes)."""
+    if "nf4_linear_gemm_kernel" in name:
+        bwd = re.search(r"NF4WCfg<\s*(true|1)", name) is not None
+        return ("bwd_gemm", "fused NF4 bwd (dX)") if bwd else ("fwd_gemm", "fused NF4 fwd (Y)")
+    if "nf4_expand_scales_kernel" in name:
+        by_col = re.search(r"nf4_expand_scales_kernel<\s*(true|1)", name) is not None
+        return ("fwd_gemm", "constants by column (fwd)") if by_col else ("bwd_gemm", "constants by row (bwd)")
+    for k in ("nf4_quantize_pass1", "nf4_mean", "nf4_dq_pass2"):
+        if k in name:
+            return "quantize", k
+    if "nf4_dequantize_kernel" in name:
+        return "dequantize", "nf4_dequantize_kernel"
+    m = re.search(r"(\w+)(<[^(]*>)?\(", name.replace("void ", "").replace("qnf4::", ""))
+    return None, (m.group(1) if m else name[:60])
+
+
+def ncu_summary(csv_path: str, last: int, calls_per_class: int, command: str) -> int:
+    """Per-kernel share of device time and DRAM bytes from an ncu launch list (metrics
+    gpu__time_duration.sum, dram__bytes_read.sum, dram__bytes_write.sum; one pass per launch) over its last
+    `last` launches, and profiles/traffic.json: DRAM bytes per timed call of each class (`calls_per_class`
+    calls of each class in those launches)."""
+    import csv
+    rows = list(csv.reader(open(csv_path)))
+    hi = next(i for i, r in enumerate(rows) if "Kernel Name" in r)
+    hdr = rows[hi]
+    ii, ki, mi, ui, vi = (hdr.index(c) for c in ("ID", "Kernel Name", "Metric Name", "Metric Unit", "Metric Value"))
+    scale = {"ns": 1e-3, "nsecond": 1e-3, "us": 1.0, "usecond": 1.0, "ms": 1e3, "msecond": 1e3, "byte": 1.0,
+             "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+    launches = {}
+    for r in rows[hi + 1:]:
+        if len(r) <= vi:
+            continue
+        d = launches.setdefault(int(r[ii]), {"name": r[ki]})
+        d[r[mi]] = float(r[vi].replace(",", "")) * scale[r[ui]]
+    sel = [launches[k] for k in sorted(launches)][-last:]
+    agg, cls_bytes = {}, {}
+    for d in sel:
+        cls, label = kernel_class(d["name"])
+        key = f"{label} [{cls}]" if cls else label
+        a = agg.setdefault(key, [0, 0.0, 0.0, 0.0])
+        rd, wr = d.get("dram__bytes_read.sum", 0.0), d.get("dram__bytes_write.sum", 0.0)
+        a[0] += 1; a[1] += d.get("gpu__time_duration.sum", 0.0); a[2] += rd; a[3] += wr
+        if cls:
+            cls_bytes[cls] = cls_bytes.get(cls, 0.0) + rd + wr
+    tot = sum(v[1] for v in agg.values())
+    print(f"{len(sel)} launches, {tot:.1f} us total")
+    print(f"{'share':>7} {'launches':>8} {'total us':>10} {'us/launch':>10} {'DRAM rd MB':>11} {'DRAM wr MB':>11}  kernel"
+          "  (DRAM per launch)")
+    for k, (n, t, rd, wr) in sorted(agg.items(), key=lambda x: -x[1][1]):
+        print(f"{t / tot * 100:6.2f}% {n:8d} {t:10.1f} {t / n:10.1f} {rd / n / 1e6:11.1f} {wr / n / 1e6:11.1f}  {k}")
+    out = {cls: {"bytes_per_launch": round(b / calls_per_class), "source_hash": source_hash(cls),
+                 "calls": calls_per_class, "command": command} for cls, b in cls_bytes.items()}
+    with open(os.path.join(ROOT, "profiles", "traffic.json"), "w") as f:
+        json.dump(out, f, indent=1)
+    for cls, e in out.items():
+        print(f"# {cls}: {e['bytes_per_launch'] / 1e6:.1f} MB of DRAM traffic per timed call")
+    return 0
 
 
 def roofline(prof: dict, steps: int, peaks: dict, peak_kind: str):
@@ -865,6 +938,11 @@ def main(argv=None):
                                            "llama65b_train", "codebook_study"],
                     default="llama7b_step",
                     help="llama7b_step (the headline line), or the decode / codec-sweep / 65B-step measurement lines")
+    ap.add_argument("--ncu-summary", metavar="CSV", default=None,
+                    help="summarise an ncu launch list (time + DRAM bytes per launch) and write profiles/traffic.json")
+    ap.add_argument("--ncu-last", type=int, default=96, help="with --ncu-summary: launches to summarise (the last N)")
+    ap.add_argument("--ncu-calls", type=int, default=6, help="with --ncu-summary: timed calls of each class in them")
+    ap.add_argument("--ncu-command", default="", help="with --ncu-summary: the command the list came from")
     ap.add_argument("--shapes", default="all",
                     help="comma-separated NxK subset of the workload shapes (profiling runs), e.g. 4096x4096")
     args = ap.parse_args(argv)
@@ -873,6 +951,8 @@ def main(argv=None):
         SHAPES = [tuple(int(v) for v in sh.split("x")) for sh in args.shapes.split(",")]
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.ncu_summary:
+        return ncu_summary(args.ncu_summary, args.ncu_last, args.ncu_calls, args.ncu_command)
     if args.impl == "reference":
         return run_reference(args)
     if args.workload == "decode":

@@ -16,6 +16,7 @@
 
 #include "qlora_nf4.h"
 #include "codec.cuh"
+#include "codebook_study.cuh"
 #include "gemm_nf4w.cuh"
 #include "gemm_sm100.cuh"
 #include "gemv_nf4.cuh"

@@ -525,136 +525,4 @@ __global__ void __launch_bounds__(256) nf4_expand_scales_kernel(const uint8_t* _
   }
 }
 
-
-// ------------------------------------------------------------------------------------------------
-// Codebook comparison (PEFT page, zerotofrontier.app/sft/peft, "NF4, derived from normal quantiles": a
-// Gaussian matrix in blocks of 64 under several codebooks, with code entropy, RMS error and Lloyd's
-// algorithm). The quantizer and the dequantizer above take any sorted codebook of 2..16 levels; these two
-// kernels measure what a codebook did to a tensor:
-//   per level j  count_j = #{elements with code j},  sum_j = sum of u = w / a (fp64, correctly rounded;
-//                0 in a block with a = 0) over those elements;
-//   overall      sse = sum of (w_hat - w)^2 in fp64, w_hat = RN32(q[code] * a) (what the dequantizer
-//                writes in fp32), and from these the code entropy in bits, the RMS error and the Lloyd
-//                update of the levels, q_j <- RN32(sum_j / count_j) (unchanged where count_j = 0).
-// Every lane sums its own elements in order, warps combine by a fixed shuffle tree, a CTA by warp order and
-// the final kernel by CTA order, so a result depends only on the input and the grid.
-// ------------------------------------------------------------------------------------------------
-constexpr int kStatThreads = 256;
-constexpr int kStatVals = 33;          // 16 counts, 16 sums of u, the squared-error sum
-constexpr int kStatMaxCtas = 1024;
-constexpr int kStatOut = 51;           // counts[16], sums[16], sse, entropy, rms, levels after one Lloyd step[16]
-
-template <typename InT>
-__global__ void __launch_bounds__(kStatThreads, 2) codebook_stats_partial(const InT* __restrict__ w,
-                                                                      const uint8_t* __restrict__ codes,
-                                                                      const float* __restrict__ absmax, int64_t n,
-                                                                      CodebookArg cb, double* __restrict__ partial) {
-  __shared__ double red[kStatThreads / 32][kStatVals];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const float qreg = cb.levels[lane & 15];
-  double sum[16];
-  uint32_t cnt[16];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) { sum[j] = 0.0; cnt[j] = 0u; }
-  double sse = 0.0;
-  const int64_t nsteps = (n + kStepElems - 1) / kStepElems;
-  const int64_t nbytes = (n + 1) / 2;
-  for (int64_t st = static_cast<int64_t>(blockIdx.x) * (kStatThreads / 32) + warp; st < nsteps;
-       st += static_cast<int64_t>(gridDim.x) * (kStatThreads / 32)) {
-    const int64_t e0 = st * kStepElems + 16 * lane;    // this lane: 16 elements of block e0 / 64
-    const bool full = (st + 1) * kStepElems <= n;
-    float x[16];
-    uint32_t c0 = 0u, c1 = 0u;
-    if (full) {
-      Raw16<InT> r;
-      r.load(w + e0);
-      r.widen(x);
-      const uint2 cc = *reinterpret_cast<const uint2*>(codes + (e0 >> 1));
-      c0 = cc.x;
-      c1 = cc.y;
-    } else {
-#pragma unroll
-      for (int e = 0; e < 16; ++e) x[e] = (e0 + e < n) ? Scalar<InT>::load(w + e0 + e) : 0.0f;
-#pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        const int64_t ib = (e0 >> 1) + b;
-        const uint32_t v = (ib < nbytes) ? codes[ib] : 0u;
-        if (b < 4) c0 |= v << (8 * b);
-        else c1 |= v << (8 * (b - 4));
-      }
-    }
-    const float a = (e0 < n) ? absmax[e0 / kBlock] : 0.0f;
-    const double ad = a;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const uint32_t byte = ((e < 8 ? c0 : c1) >> (8 * ((e >> 1) & 3))) & 0xFFu;
-      const uint32_t code = (e & 1) ? (byte & 0xFu) : (byte >> 4);
-      const float q = lut16(qreg, code);                                   // the whole warp takes part
-      const bool valid = full || (e0 + e < n);
-      const double xd = x[e];
-      const double u = (a > 0.0f) ? xd / ad : 0.0;
-      const double d = __dsub_rn(static_cast<double>(__fmul_rn(q, a)), xd);
-      if (valid) sse = __dadd_rn(sse, __dmul_rn(d, d));
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const bool hit = valid && code == static_cast<uint32_t>(j);
-        sum[j] += hit ? u : 0.0;
-        cnt[j] += hit ? 1u : 0u;
-      }
-    }
-  }
-  // warp: fixed xor tree; CTA: warp order
-  double v[kStatVals];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) { v[j] = static_cast<double>(cnt[j]); v[16 + j] = sum[j]; }
-  v[32] = sse;
-#pragma unroll
-  for (int k = 0; k < kStatVals; ++k) {
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) v[k] += __shfl_xor_sync(0xffffffffu, v[k], off);
-  }
-  if (lane == 0) {
-#pragma unroll
-    for (int k = 0; k < kStatVals; ++k) red[warp][k] = v[k];
-  }
-  __syncthreads();
-  if (threadIdx.x < kStatVals) {
-    double t = 0.0;
-    for (int wi = 0; wi < kStatThreads / 32; ++wi) t += red[wi][threadIdx.x];
-    partial[static_cast<int64_t>(blockIdx.x) * kStatVals + threadIdx.x] = t;
-  }
-}
-
-__global__ void __launch_bounds__(64) codebook_stats_final(const double* __restrict__ partial, int nctas, int64_t n,
-                                                          CodebookArg cb, int nlevels, double* __restrict__ out) {
-  __shared__ double tot[kStatVals];
-  const int t = threadIdx.x;
-  if (t < kStatVals) {
-    double s = 0.0;
-    for (int g = 0; g < nctas; ++g) s += partial[static_cast<int64_t>(g) * kStatVals + t];
-    tot[t] = s;
-  }
-  __syncthreads();
-  if (t < 16) {
-    out[t] = tot[t];
-    out[16 + t] = tot[16 + t];
-    const bool used = t < nlevels && tot[t] > 0.0;
-    out[35 + t] = used ? static_cast<double>(static_cast<float>(tot[16 + t] / tot[t]))
-                       : static_cast<double>(cb.levels[t]);
-  }
-  if (t == 0) {
-    const double nd = static_cast<double>(n);
-    double h = 0.0;
-    for (int j = 0; j < 16; ++j) {
-      if (tot[j] > 0.0) {
-        const double p = tot[j] / nd;
-        h -= p * log2(p);
-      }
-    }
-    out[32] = tot[32];
-    out[33] = h;
-    out[34] = sqrt(tot[32] / nd);
-  }
-}
-
 }  // namespace qnf4

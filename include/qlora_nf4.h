@@ -191,7 +191,8 @@ int qlora_nf4_dequantize_single(const void* codes, const float* absmax, int64_t 
  *                              qlora_codebook_quantize with the same levels; w finite). `stats` is a
  *                              device array of QLORA_CODEBOOK_STATS_LEN doubles:
  *       [0..15]   count_j, the number of elements with code j
- *       [16..31]  sum_j, the sum of u = w / a (fp64, correctly rounded; 0 in an all-zero block) over them
+ *       [16..31]  sum_j, the sum of u = w / a over them in fp64 (u formed as w * fp64(1/a), within one
+ *                 fp64 ulp of the quotient; 0 in an all-zero block)
  *       [32]      sum over all elements of (w_hat - w)^2 in fp64, w_hat as qlora_codebook_dequantize's fp32
  *       [33]      code entropy in bits, -sum_j p_j log2 p_j with p_j = count_j / n
  *       [34]      RMS error, sqrt([32] / n)
