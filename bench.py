@@ -672,6 +672,8 @@ def run_codebook_study(args):
     st = torch.empty(q.CODEBOOK_STATS_LEN, dtype=torch.float64, device=device)
     ws = torch.empty(q.codebook_stats_workspace_bytes(n), dtype=torch.uint8, device=device)
     stored = 0.5 + 4 / 64
+    for _ in range(args.warmup):
+        q.lloyd(x, nf4, 1)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
