@@ -18,6 +18,8 @@ What it computes, in the pages' order (citations are to the source pages by titl
   codebook_study.py  the codebook comparison: any sorted codebook of up to 16 levels with fp32 block
                constants, code entropy and RMS error, and Lloyd's algorithm
                [PEFT page, "NF4, derived from normal quantiles"]
+  adamw.py     the AdamW step whose states the paged optimizer keeps in unified memory
+               [PEFT page, "Paged optimizers, and QLoRA end to end"]
   linear.py    the QLoRA linear layer, forward and backward, in fp64
                [QLoRA explainer, prism.theerrors.in, "Putting it together";
                 PEFT page, "Paged optimizers, and QLoRA end to end"]
@@ -35,5 +37,6 @@ from .codec import (BLOCK, DQ_BLOCK, num_blocks, num_groups, storage_bytes, absm
                     quantize_single, dequantize_single, storage_bytes_single, NF4SingleTensor)
 from .linear import linear_fwd, linear_bwd
 from . import codebook_study
+from .adamw import adamw_step
 
 __all__ = [n for n in dir() if not n.startswith("_")]
