@@ -9,6 +9,7 @@ include/qlora_nf4.h:
     linear_fwd(X, q, A, B, alpha)    -> (Y, U)        (qlora_linear_fwd)
     linear_bwd(dY, X, q, A, B, alpha, U) -> (dX, dA, dB)   (qlora_linear_bwd)
     codebook_quantize / codebook_dequantize / codebook_stats   (qlora_codebook_*)
+    adamw_step, paged_empty, paged_prefetch   (qlora_adamw_step, qlora_paged_*; optim.PagedAdamW)
 
 The shared library is loaded on first use (so that the build step, a submodule of this package, can run
 before it exists); a call made while it is not built raises ImportError. There is no fallback
@@ -73,6 +74,11 @@ def _open() -> ctypes.CDLL:
         "qlora_codebook_dequantize": [vp, vp, i64, P(ctypes.c_float), i32, vp, i32, vp],
         "qlora_codebook_stats_workspace": [i64, P(sz)],
         "qlora_codebook_stats": [vp, i32, vp, vp, i64, P(ctypes.c_float), i32, vp, vp, sz, vp],
+        "qlora_adamw_step": [vp, vp, vp, vp, vp, i64, i64, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                             ctypes.c_float, ctypes.c_float, vp],
+        "qlora_paged_alloc": [sz, P(vp)],
+        "qlora_paged_free": [vp],
+        "qlora_paged_prefetch": [vp, sz, i32, vp],
         "qlora_linear_workspace": [i64, i64, i64, i32, P(sz)],
         "qlora_linear_fwd": [vp, i64, P(_NF4Struct), vp, vp, i32, ctypes.c_float, vp, vp, vp, sz, vp],
         "qlora_linear_bwd": [vp, vp, i64, P(_NF4Struct), vp, vp, i32, ctypes.c_float, vp, vp, vp, vp,
@@ -314,6 +320,56 @@ def lloyd(w: torch.Tensor, levels, iters: int, stream=None):
         if k < iters:
             lv = d["centroids"]
     return lv, hist
+
+
+# ---- paged optimizer: AdamW step and managed-memory buffers ------------------------------------------
+
+def adamw_step(p: torch.Tensor, g: torch.Tensor, m: torch.Tensor, v: torch.Tensor, step: int, lr: float,
+               betas=(0.9, 0.999), eps: float = 1e-8, weight_decay: float = 0.0,
+               p_bf16: torch.Tensor | None = None, stream=None) -> None:
+    """qlora_adamw_step on contiguous fp32 CUDA tensors of equal size (device or managed memory)."""
+    n = p.numel()
+    for t, name in ((p, "p"), (g, "g"), (m, "m"), (v, "v")):
+        if t.dtype != torch.float32 or not t.is_contiguous() or t.numel() != n:
+            raise ValueError(f"adamw_step: {name} must be a contiguous float32 tensor of {n} elements")
+    if p_bf16 is not None and (p_bf16.dtype != torch.bfloat16 or p_bf16.numel() != n or not p_bf16.is_contiguous()):
+        raise ValueError("adamw_step: p_bf16 must be a contiguous bfloat16 tensor of the same size")
+    _check(load().qlora_adamw_step(_ptr(p), _ptr(g), _ptr(m), _ptr(v), _ptr(p_bf16), n, int(step), lr, betas[0],
+                                   betas[1], eps, weight_decay, _stream(stream)), "qlora_adamw_step")
+
+
+class PagedBuffer:
+    """Managed memory from qlora_paged_alloc, freed with qlora_paged_free when the last tensor viewing it
+    goes away; exposes __cuda_array_interface__ so torch.as_tensor can wrap it without a copy."""
+
+    def __init__(self, n: int, device=None):
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.device = dev
+        self.n = int(n)
+        self.nbytes = 4 * self.n
+        self.ptr = ctypes.c_void_p()
+        with torch.cuda.device(dev):
+            _check(load().qlora_paged_alloc(self.nbytes, ctypes.byref(self.ptr)), "qlora_paged_alloc")
+        self.__cuda_array_interface__ = {"shape": (self.n,), "typestr": "<f4", "data": (self.ptr.value, False),
+                                         "version": 3, "strides": None}
+
+    def __del__(self):
+        if getattr(self, "ptr", None) is not None and self.ptr.value:
+            load().qlora_paged_free(self.ptr)
+            self.ptr = ctypes.c_void_p()
+
+
+def paged_empty(n: int, device=None) -> torch.Tensor:
+    """An n-element float32 tensor in managed (unified) memory; uninitialised."""
+    buf = PagedBuffer(n, device)
+    with torch.cuda.device(buf.device):
+        return torch.as_tensor(buf, device=buf.device)
+
+
+def paged_prefetch(t: torch.Tensor, to_device: bool = True, stream=None) -> None:
+    """Migrate a managed-memory tensor's pages to the GPU, or to host memory (an eviction)."""
+    _check(load().qlora_paged_prefetch(_ptr(t), t.numel() * t.element_size(), 1 if to_device else 0, _stream(stream)),
+           "qlora_paged_prefetch")
 
 
 NOALLOC_MAX_NUMEL = 1 << 26

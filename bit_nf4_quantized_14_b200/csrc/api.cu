@@ -17,6 +17,7 @@
 #include "qlora_nf4.h"
 #include "codec.cuh"
 #include "codebook_study.cuh"
+#include "adamw.cuh"
 #include "gemm_nf4w.cuh"
 #include "gemm_sm100.cuh"
 #include "gemv_nf4.cuh"
@@ -833,6 +834,68 @@ int qlora_codebook_stats(const void* w, int w_dtype, const void* codes, const fl
   if (int e = launched()) return e;
   codebook_stats_final<<<1, 64, 0, st>>>(part, static_cast<int>(G), n, cb, nlevels, stats);
   return launched();
+}
+
+int qlora_adamw_step(float* p, const float* g, float* m, float* v, void* p_bf16, int64_t n, int64_t step, float lr,
+                     float beta1, float beta2, float eps, float weight_decay, qlora_stream_t stream) {
+  if (!p || !g || !m || !v) return QLORA_ERR_INVALID_ARG;
+  if (step < 1 || !(lr >= 0.0f) || !(lr < INFINITY) || !(beta1 >= 0.0f && beta1 < 1.0f) ||
+      !(beta2 >= 0.0f && beta2 < 1.0f) || !(eps > 0.0f && eps < INFINITY) || !(weight_decay >= 0.0f) ||
+      !(weight_decay < INFINITY))
+    return QLORA_ERR_INVALID_ARG;
+  if (n <= 0 || n > kMaxNumel) return QLORA_ERR_SHAPE;
+  if (!aligned16(p) || !aligned16(g) || !aligned16(m) || !aligned16(v) || !aligned16(p_bf16)) return QLORA_ERR_ALIGNMENT;
+  int sms = 0;
+  if (int e = check_device(&sms)) return e;
+  AdamWArgs a;
+  const double t = static_cast<double>(step);
+  a.keep = static_cast<float>(1.0 - static_cast<double>(lr) * weight_decay);
+  a.beta1 = beta1;
+  a.one_minus_beta1 = static_cast<float>(1.0 - beta1);
+  a.beta2 = beta2;
+  a.one_minus_beta2 = static_cast<float>(1.0 - beta2);
+  a.step_size = static_cast<float>(lr / (1.0 - std::pow(static_cast<double>(beta1), t)));
+  a.inv_bc2_sqrt = static_cast<float>(1.0 / std::sqrt(1.0 - std::pow(static_cast<double>(beta2), t)));
+  a.eps = eps;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const unsigned grid = static_cast<unsigned>(
+      std::max<int64_t>(1, std::min<int64_t>(cdiv(n / 4, kAdamThreads), int64_t(sms) * 8)));
+  if (p_bf16)
+    adamw_kernel<true><<<grid, kAdamThreads, 0, st>>>(p, g, m, v, static_cast<__nv_bfloat16*>(p_bf16), n, a);
+  else
+    adamw_kernel<false><<<grid, kAdamThreads, 0, st>>>(p, g, m, v, nullptr, n, a);
+  return launched();
+}
+
+int qlora_paged_alloc(size_t bytes, void** ptr) {
+  if (!ptr || bytes == 0) return QLORA_ERR_INVALID_ARG;
+  *ptr = nullptr;
+  if (int e = check_device(nullptr)) return e;
+  if (cudaMallocManaged(ptr, bytes, cudaMemAttachGlobal) != cudaSuccess) {
+    *ptr = nullptr;
+    return cuda_fail(cudaGetLastError(), "cudaMallocManaged", __LINE__);
+  }
+  return QLORA_OK;
+}
+
+int qlora_paged_free(void* ptr) {
+  if (!ptr) return QLORA_OK;
+  if (cudaFree(ptr) != cudaSuccess) return cuda_fail(cudaGetLastError(), "cudaFree", __LINE__);
+  return QLORA_OK;
+}
+
+int qlora_paged_prefetch(const void* ptr, size_t bytes, int to_device, qlora_stream_t stream) {
+  if (!ptr || bytes == 0) return QLORA_ERR_INVALID_ARG;
+  if (int e = check_device(nullptr)) return e;
+  int dev = 0, concurrent = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&concurrent, cudaDevAttrConcurrentManagedAccess, dev) != cudaSuccess)
+    return cuda_fail(cudaGetLastError(), "cudaDeviceGetAttribute", __LINE__);
+  if (!concurrent) return QLORA_ERR_UNSUPPORTED;
+  if (cudaMemPrefetchAsync(ptr, bytes, to_device ? dev : cudaCpuDeviceId, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return cuda_fail(cudaGetLastError(), "cudaMemPrefetchAsync", __LINE__);
+  return QLORA_OK;
 }
 
 int qlora_linear_workspace(int64_t T, int64_t N, int64_t K, int r, size_t* bytes) {

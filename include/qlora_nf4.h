@@ -14,7 +14,8 @@
  *
  * Conventions for every call:
  *   - All tensor pointers are DEVICE pointers unless a parameter says "host". The caller owns and
- *     allocates every buffer; the library never allocates device memory and keeps no per-call state.
+ *     allocates every buffer; the library never allocates device memory and keeps no per-call state
+ *     (the one exception is qlora_paged_alloc, which allocates managed memory on request).
  *     Its only state is a constant-memory codebook and one status word per device.
  *   - Every device pointer must be 16-byte aligned (QLORA_ERR_ALIGNMENT otherwise).
  *   - Layouts are row-major and dense. bf16 tensors are passed as `const void*`/`void*`.
@@ -210,6 +211,35 @@ int qlora_codebook_stats_workspace(int64_t n, size_t* bytes);
 int qlora_codebook_stats(const void* w, int w_dtype, const void* codes, const float* absmax, int64_t n,
                          const float* levels, int nlevels, double* stats, void* workspace,
                          size_t workspace_bytes, qlora_stream_t stream);
+
+/*
+ * Paged optimizer [PEFT "Paged optimizers, and QLoRA end to end": the optimizer states are allocated in
+ * NVIDIA unified memory, which the driver pages between GPU and CPU RAM when the GPU runs short, and paged
+ * back when the optimizer step needs them; EXPL "The three innovations": paged optimizers absorb memory
+ * spikes]. The update is not written on the pages; it is the standard AdamW (Adam with decoupled weight
+ * decay, Loshchilov & Hutter 2019) in fp32:
+ *     p <- p (1 - lr wd);  m <- b1 m + (1 - b1) g;  v <- b2 v + (1 - b2) g^2;
+ *     p <- p - [lr / (1 - b1^t)] m / (sqrt(v) / sqrt(1 - b2^t) + eps)
+ * with the two bias corrections formed in fp64 on the host for step t >= 1.
+ *
+ * qlora_adamw_step   one fused pass over n fp32 elements: p (read, written), g (read), m and v (read,
+ *                    written); p_bf16 (n bf16, or NULL) receives bf16(p) after the update. The pointers may
+ *                    be device memory or managed memory from qlora_paged_alloc, resident or not (pages move
+ *                    to the GPU as the kernel touches them). QLORA_ERR_INVALID_ARG unless t >= 1,
+ *                    0 <= b1, b2 < 1, eps > 0, lr >= 0 and wd >= 0 (all finite).
+ * qlora_paged_alloc  *ptr = `bytes` of managed (unified) memory, accessible from the host and every GPU;
+ *                    contents uninitialised. The one call that allocates: the caller frees with
+ *                    qlora_paged_free.
+ * qlora_paged_prefetch  enqueue on `stream` a migration of [ptr, ptr + bytes) to the current GPU
+ *                    (to_device != 0) or to host memory (to_device == 0, as the driver does when it evicts
+ *                    under memory pressure). QLORA_ERR_UNSUPPORTED if the GPU cannot access managed memory
+ *                    concurrently with the host.
+ */
+int qlora_adamw_step(float* p, const float* g, float* m, float* v, void* p_bf16, int64_t n, int64_t step,
+                     float lr, float beta1, float beta2, float eps, float weight_decay, qlora_stream_t stream);
+int qlora_paged_alloc(size_t bytes, void** ptr);
+int qlora_paged_free(void* ptr);
+int qlora_paged_prefetch(const void* ptr, size_t bytes, int to_device, qlora_stream_t stream);
 
 /*
  * Device workspace bytes for qlora_linear_fwd / qlora_linear_bwd with T tokens, weight N x K (out x in)

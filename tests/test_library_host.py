@@ -152,3 +152,25 @@ def test_codebook_calls_reject_bad_codebooks_before_any_cuda_call(q):
     b = ctypes.c_size_t()
     assert L.qlora_codebook_stats_workspace(1 << 30, ctypes.byref(b)) == 0 and b.value >= 33 * 8
     assert L.qlora_codebook_stats_workspace(0, ctypes.byref(b)) == -2
+
+
+def test_adamw_and_paged_calls_reject_bad_arguments_before_any_cuda_call(q):
+    L = q.lib
+    P, G, M, Vv = V(0x300000), V(0x310000), V(0x320000), V(0x330000)
+    ok = dict(step=1, lr=2e-4, b1=0.9, b2=0.999, eps=1e-8, wd=0.0)
+
+    def call(p=P, n=64, **kw):
+        a = dict(ok, **kw)
+        return L.qlora_adamw_step(p, G, M, Vv, None, n, a["step"], a["lr"], a["b1"], a["b2"], a["eps"], a["wd"], None)
+
+    assert call(p=None) == -1
+    assert call(step=0) == -1
+    assert call(lr=float("nan")) == -1 and call(lr=-1.0) == -1 and call(lr=float("inf")) == -1
+    assert call(b1=1.0) == -1 and call(b2=-0.1) == -1
+    assert call(eps=0.0) == -1 and call(wd=-0.5) == -1
+    assert call(n=0) == -2
+    assert call(p=V(0x300004)) == -3
+    assert L.qlora_paged_alloc(0, ctypes.byref(V())) == -1
+    assert L.qlora_paged_alloc(64, None) == -1
+    assert L.qlora_paged_prefetch(None, 64, 1, None) == -1
+    assert L.qlora_paged_free(None) == 0
