@@ -983,6 +983,9 @@ def run_llama65b_train(args):
     def step():
         if args.optimizer == "paged_evicted":
             opt.evict_states()          # a memory spike pushed the moments out; the step pages them back
+        elif args.optimizer == "paged_evicted_prefetch":
+            opt.prefetch_states_async(evict_first=True)   # the same spike, then the moments are brought
+                                                          # back while the forward and backward run
         loss = model(ids, targets)
         loss.backward()
         opt.step()
@@ -1026,7 +1029,10 @@ def run_llama65b_train(args):
                       "optimizer": {"torch": "torch.optim.AdamW (fused, device states)",
                                     "paged": "PagedAdamW (library kernel, moments in managed memory, resident)",
                                     "paged_evicted": "PagedAdamW, moments evicted to the host at the start of every "
-                                                     "step and paged back by the optimizer step"}[args.optimizer],
+                                                     "step and paged back by the optimizer step",
+                                    "paged_evicted_prefetch": "PagedAdamW, moments evicted at the start of every "
+                                                              "step on a side stream and prefetched back there "
+                                                              "while the forward and backward run"}[args.optimizer],
                       "library_linears_ms_per_step": round(lin_ms, 3),
                       "library_linears_share": round(lin_ms / ms, 4),
                       "final_loss": float(loss.item()), "gpu_launches": int(launches), "clocks": clk,
@@ -1042,7 +1048,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) measurement")
-    ap.add_argument("--optimizer", choices=["torch", "paged", "paged_evicted"], default="torch",
+    ap.add_argument("--optimizer", choices=["torch", "paged", "paged_evicted", "paged_evicted_prefetch"],
+                    default="torch",
                     help="with --workload llama65b_train: the adapters' optimizer")
     ap.add_argument("--workload", choices=["llama7b_step", "decode", "codec_sweep", "llama65b_linears",
                                            "llama65b_train", "codebook_study", "paged_adamw"],

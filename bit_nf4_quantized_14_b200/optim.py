@@ -9,6 +9,8 @@ Argument marshalling and buffer bookkeeping only: the update runs in the library
 """
 from __future__ import annotations
 
+import threading
+
 import torch
 
 from . import adamw_step, paged_empty, paged_prefetch
@@ -45,12 +47,20 @@ class PagedAdamW:
         self.m.zero_()
         self.v.zero_()
         self.t = 0
+        self._side = None
+        self._ready = None
+        self._thread = None
 
     def zero_grad(self) -> None:
         """Zero the gradients in place (they are views of one flat buffer that autograd adds into)."""
         self.flat_g.zero_()
 
     def step(self, stream=None) -> None:
+        if self._ready is not None:            # moments still on their way back: wait on the device
+            self._thread.join()
+            (stream if stream is not None else torch.cuda.current_stream()).wait_event(self._ready)
+            self._ready = None
+            self._thread = None
         self.t += 1
         adamw_step(self.flat_p, self.flat_g, self.m, self.v, self.t, self.lr, self.betas, self.eps,
                    self.weight_decay, stream=stream)
@@ -68,6 +78,37 @@ class PagedAdamW:
             return
         paged_prefetch(self.m, True, stream)
         paged_prefetch(self.v, True, stream)
+
+    def side_stream(self) -> torch.cuda.Stream:
+        if self._side is None:
+            self._side = torch.cuda.Stream(device=self.flat_p.device)
+        return self._side
+
+    def prefetch_states_async(self, evict_first: bool = False) -> None:
+        """Bring the moments back to the GPU on a side stream, issued from a worker thread (a migration
+        call can hold the calling thread while the driver moves pages), so that it overlaps whatever the
+        current stream runs next -- the forward and backward passes; the next step() waits for it.
+        evict_first moves them to the host first, as the driver does under a memory spike (to measure
+        the cost of paging)."""
+        if not self.paged:
+            return
+        side = self.side_stream()
+        side.wait_stream(torch.cuda.current_stream())
+        ready = torch.cuda.Event()
+        dev = self.flat_p.device
+
+        def work():
+            torch.cuda.set_device(dev)
+            if evict_first:
+                paged_prefetch(self.m, False, side)
+                paged_prefetch(self.v, False, side)
+            paged_prefetch(self.m, True, side)
+            paged_prefetch(self.v, True, side)
+            ready.record(side)
+
+        self._thread = threading.Thread(target=work, daemon=True)
+        self._thread.start()
+        self._ready = ready
 
     def state_bytes(self) -> int:
         return 8 * self.n

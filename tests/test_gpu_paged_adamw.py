@@ -11,6 +11,16 @@ import synth
 pytestmark = pytest.mark.gpu
 
 
+def f32(x):
+    """The value the library receives for a float argument."""
+    return float(np.float32(x))
+
+
+def oracle(p, g, m, v, t, lr, wd):
+    """The oracle step with the hyper-parameters as the fp32 values the kernel is given."""
+    return oracle_step(p, g, m, v, t, f32(lr), beta1=f32(0.9), beta2=f32(0.999), eps=f32(1e-8), wd=f32(wd))
+
+
 def _bounds_ok(p_new, m_new, v_new, ref, p_old, g, m_old, v_old, t, lr):
     """fp32 evaluation of one step against the exact fp64 step from the same fp32 inputs: a few roundings
     of each term (m may cancel, so its bound is on the terms, not on the sum)."""
@@ -43,7 +53,7 @@ def _run_steps(lib, n, steps, wd, make_state, evict=False):
         torch.cuda.synchronize()
         pn, mn, vn = p.cpu().numpy(), m.cpu().numpy(), v.cpu().numpy()
         gn = g.cpu().numpy()
-        ref = oracle_step(p0, gn, m0, v0, t, lr, wd=wd)
+        ref = oracle(p0, gn, m0, v0, t, lr, wd)
         _bounds_ok(pn, mn, vn, ref, p0, gn, m0, v0, t, lr)
         assert torch.equal(p16.cpu(), p.cpu().to(torch.bfloat16)), "bf16 copy"
         hist.append((pn.copy(), mn.copy(), vn.copy()))
@@ -89,6 +99,8 @@ def test_paged_adamw_on_qlora_layers(lib):
         opt.zero_grad()
         if t == 3:
             opt.evict_states()
+        if t == 4:
+            opt.prefetch_states_async(evict_first=True)
         loss = ((l2(l1(x)).float() - target) ** 2).mean()
         loss.backward()
         p0 = opt.flat_p.cpu().numpy().copy()
@@ -97,9 +109,9 @@ def test_paged_adamw_on_qlora_layers(lib):
         assert np.any(g != 0)
         opt.step()
         torch.cuda.synchronize()
-        ref = oracle_step(p0, g, m0, v0, t, 1e-3, wd=0.01)
+        ref = oracle(p0, g, m0, v0, t, 1e-3, 0.01)
         _bounds_ok(opt.flat_p.cpu().numpy(), opt.m.cpu().numpy(), opt.v.cpu().numpy(), ref, p0, g, m0, v0, t, 1e-3)
         # the parameters the layers see are the updated flat buffer
         assert torch.equal(l2.B.detach().reshape(-1).cpu(), opt.flat_p[-l2.B.numel():].cpu())
-        losses.append(float(loss))
+        losses.append(float(loss.detach()))
     assert losses[-1] < losses[0]
