@@ -240,12 +240,11 @@ bool tmap_mnmajor(CUtensorMap* m, const void* p, uint64_t mn, uint64_t contracti
 
 // ---- GEMM launches ------------------------------------------------------------------------------
 template <class C>
-int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
-                const CUtensorMap& b2, const GemmParams& p, cudaStream_t st) {
+int launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, cudaStream_t st) {
   auto kern = gemm_sm100_kernel<C>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
-  kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, a2, b2, p, codebook());
+  kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(a, b, p);
   return launched();
 }
 
@@ -328,14 +327,15 @@ template <int BN, Skinny S>
 int launch_skinny(const CUtensorMap& a, const CUtensorMap& b, int64_t M, int64_t C, float* part,
                   int64_t part_stride, cudaStream_t st) {
   constexpr bool AMN = (S == Skinny::kGrad), BMN = (S != Skinny::kU);
-  using Cfg = GemmCfg<BN, AMN, BMN, BSrc::kTma, false, Epi::kF32Partial, skinny_stages<BN>()>;
+  using Cfg = GemmCfg<BN, AMN, BMN, skinny_stages<BN>()>;
   const int64_t tiles = cdiv(M, 128), nkb = cdiv(C, 64);
   const Split sp = choose_split(tiles, nkb);
   GemmParams p{};
-  p.M = static_cast<int>(M); p.N = BN;
-  p.nkb_total = static_cast<int>(nkb); p.kb_split = sp.kb_split; p.nkb2 = 0;
-  p.out = part; p.ldo = BN; p.part_stride = part_stride;
-  return launch_gemm<Cfg>(dim3(1, static_cast<unsigned>(tiles), sp.splits), a, b, a, b, p, st);
+  p.nkb_total = static_cast<int>(nkb);
+  p.kb_split = sp.kb_split;
+  p.out = part;
+  p.part_stride = part_stride;
+  return launch_gemm<Cfg>(dim3(1, static_cast<unsigned>(tiles), sp.splits), a, b, p, st);
 }
 template <Skinny S>
 int launch_skinny_bn(int bn, const CUtensorMap& a, const CUtensorMap& b, int64_t M, int64_t C, float* part,
