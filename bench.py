@@ -244,7 +244,7 @@ def kernel_class(name: str):
     return None, (m.group(1) if m else name[:60])
 
 
-def ncu_summary(csv_path: str, last: int, calls_per_class: int, command: str) -> int:
+def ncu_summary(csv_path: str, last: int, calls_per_class: int, command: str, out_path: str | None = None) -> int:
     """Per-kernel share of device time and DRAM bytes from an ncu launch list (metrics
     gpu__time_duration.sum, dram__bytes_read.sum, dram__bytes_write.sum; one pass per launch) over its last
     `last` launches, and profiles/traffic.json: DRAM bytes per timed call of each class (`calls_per_class`
@@ -280,7 +280,7 @@ def ncu_summary(csv_path: str, last: int, calls_per_class: int, command: str) ->
         print(f"{t / tot * 100:6.2f}% {n:8d} {t:10.1f} {t / n:10.1f} {rd / n / 1e6:11.1f} {wr / n / 1e6:11.1f}  {k}")
     out = {cls: {"bytes_per_launch": round(b / calls_per_class), "source_hash": source_hash(cls),
                  "calls": calls_per_class, "command": command} for cls, b in cls_bytes.items()}
-    with open(os.path.join(ROOT, "profiles", "traffic.json"), "w") as f:
+    with open(out_path or os.path.join(ROOT, "profiles", "traffic.json"), "w") as f:
         json.dump(out, f, indent=1)
     for cls, e in out.items():
         print(f"# {cls}: {e['bytes_per_launch'] / 1e6:.1f} MB of DRAM traffic per timed call")

@@ -61,3 +61,39 @@ def test_max_over_ranks_gloo_world2():
 
 def test_single_process_reduction_is_identity():
     assert bench.max_over_ranks(3.25) == 3.25
+
+
+def test_kernel_classes_of_ncu_names():
+    kc = bench.kernel_class
+    assert kc("void qnf4::nf4_linear_gemm_kernel<qnf4::NF4WCfg<false, 2>>(CUtensorMap_st, ...)")[0] == "fwd_gemm"
+    assert kc("void qnf4::nf4_linear_gemm_kernel<qnf4::NF4WCfg<true, 2>>(CUtensorMap_st, ...)")[0] == "bwd_gemm"
+    assert kc("void qnf4::nf4_linear_gemm_kernel<qnf4::NF4WCfg<1, 2>>(...)")[0] == "bwd_gemm"
+    assert kc("void qnf4::nf4_expand_scales_kernel<true>(const unsigned char *, ...)")[0] == "fwd_gemm"
+    assert kc("void qnf4::nf4_expand_scales_kernel<0>(const unsigned char *, ...)")[0] == "bwd_gemm"
+    for k in ("nf4_quantize_pass1<float>(const T1 *)", "nf4_mean(const double *)", "nf4_dq_pass2(const float *)"):
+        assert kc("void qnf4::" + k)[0] == "quantize"
+    assert kc("void qnf4::nf4_dequantize_kernel<1, 0>(const unsigned char *)")[0] == "dequantize"
+    cls, label = kc("void qnf4::gemm_sm100_kernel<qnf4::GemmCfg<64, false, false, 3>>(CUtensorMap_st)")
+    assert cls is None and label == "gemm_sm100_kernel"
+
+
+def test_ncu_summary_writes_per_call_traffic(tmp_path, capsys):
+    """A hand-made launch list: two timed calls of each class, one extra kernel outside the classes."""
+    rows = [["ID", "Kernel Name", "Metric Name", "Metric Unit", "Metric Value"]]
+    names = ["void qnf4::nf4_expand_scales_kernel<1>(x)", "void qnf4::nf4_linear_gemm_kernel<qnf4::NF4WCfg<0, 2>>(x)",
+             "void qnf4::split_reduce_kernel<0>(x)"] * 2
+    for i, n in enumerate(names):
+        rows += [[str(i), n, "gpu__time_duration.sum", "us", "10"],
+                 [str(i), n, "dram__bytes_read.sum", "Mbyte", str(1 + i)],
+                 [str(i), n, "dram__bytes_write.sum", "byte", "1000"]]
+    csv_path = tmp_path / "launches.csv"
+    csv_path.write_text("\n".join(",".join(f'"{c}"' for c in r) for r in rows) + "\n")
+    out = tmp_path / "traffic.json"
+    assert bench.ncu_summary(str(csv_path), 6, 2, "cmd", str(out)) == 0
+    import json
+    t = json.loads(out.read_text())
+    # fwd_gemm launches are ids 0, 1, 3, 4: (1 + 2 + 4 + 5) MB read + 4 x 1000 B written, over 2 calls
+    assert t["fwd_gemm"]["bytes_per_launch"] == round((12e6 + 4000) / 2)
+    assert t["fwd_gemm"]["source_hash"] == bench.source_hash("fwd_gemm") and t["fwd_gemm"]["command"] == "cmd"
+    assert set(t) == {"fwd_gemm"}
+    assert "6 launches" in capsys.readouterr().out
