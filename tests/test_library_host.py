@@ -174,3 +174,44 @@ def test_adamw_and_paged_calls_reject_bad_arguments_before_any_cuda_call(q):
     assert L.qlora_paged_alloc(64, None) == -1
     assert L.qlora_paged_prefetch(None, 64, 1, None) == -1
     assert L.qlora_paged_free(None) == 0
+
+
+def test_codebook_density_rule(q):
+    """Any codebook whose thresholds are more than one widened bucket (1/15 + 2^-17 in w / a) apart is
+    accepted; two thresholds inside one bucket are rejected. Accepted calls go on to the device check and
+    fail there without a GPU (or succeed with one), never with QLORA_ERR_CODEBOOK."""
+    from oracle import codebook_study as CS
+    import torch
+    L = q.lib
+    F = ctypes.c_float
+    W, C, A = V(0x300000), V(0x310000), V(0x320000)
+    rng = np.random.default_rng(7)
+    gap = 1 / 15 + 2.0 ** -17
+    if torch.cuda.is_available():
+        pytest.skip("the accepted calls would run on the device")
+    for _ in range(200):
+        nl = int(rng.integers(2, 17))
+        # levels whose midpoints are at least `gap` apart: spread the levels by more than that
+        steps = rng.uniform(gap * 1.01, 2.0 / max(nl - 1, 1), size=nl - 1)
+        lv = np.concatenate([[0.0], np.cumsum(steps)])
+        lv = lv - lv[-1] / 2
+        if np.abs(lv).max() > 1:
+            lv = lv / np.abs(lv).max()
+        lv = lv.astype(np.float32)
+        th = CS.thresholds(lv).astype(np.float64)
+        if len(th) > 1 and np.diff(th).min() <= gap:
+            continue
+        arr = (F * nl)(*lv.tolist())
+        assert L.qlora_codebook_quantize(W, 0, 4096, arr, nl, C, A, None) != -10, lv
+    rejected = 0
+    for centre in np.linspace(-0.9, 0.9, 19):
+        # two thresholds 0.01 apart around the centre b of a bucket (buckets are 1/15 wide): levels
+        # l0 = m0 - d, l1 = m0 + d, l2 = 2 m1 - l1 have midpoints m0 and m1
+        b = round(centre * 15) / 15
+        m0, m1, d = b - 0.005, b + 0.005, 0.004
+        lv = np.array([m0 - d, m0 + d, 2 * m1 - (m0 + d)], np.float32)
+        assert np.all(np.diff(lv) > 0) and np.abs(lv).max() <= 1
+        arr = (F * 3)(*lv.tolist())
+        assert L.qlora_codebook_quantize(W, 0, 4096, arr, 3, C, A, None) == -10, lv
+        rejected += 1
+    assert rejected == 19
