@@ -229,3 +229,42 @@ def test_single_variant_special_values(lib):
     x = np.concatenate([np.zeros(128, np.float32), np.float32([1e-40, -3e-39] + [0.0] * 62),
                         np.float32([3e38, -1e38] + [1e30] * 62), synth.normal_f32(64 * 50 + 3, 0.02, 0, 77)])
     _assert_single_same(lib, torch.from_numpy(x).cuda(), O.quantize_single(x), x.size)
+
+
+def test_largest_sweep_size_2_31(lib):
+    """The top of the quantize/dequantize size sweep, 2^31 elements (eight 2^28-element sweep tensors,
+    drawn as the benchmark draws them; indices past 2^31 - 1 exercise 64-bit addressing): every block
+    constant's E4M3 value, every group scale and the mean exact against the oracle, and the codes and
+    dequantized bf16 values of 4096 sampled blocks."""
+    n, chunk = 1 << 31, 1 << 28
+    dev = torch.device("cuda", 0)
+    x = torch.empty(n, dtype=torch.float32, device=dev)
+    c1 = np.empty(n // 64, np.float32)
+    sb = np.sort(np.random.default_rng(1).choice(n // 64, 4096, replace=False))
+    sv = np.empty((sb.size, 64), np.float32)
+    for c in range(0, n, chunk):
+        xc = synth.sweep_f32(chunk, seed=50, tensor_id=c // chunk)
+        x[c:c + chunk] = torch.from_numpy(xc).to(dev)
+        c1[c // 64:(c + chunk) // 64] = O.absmax_blocks(xc)
+        for i in np.nonzero((sb >= c // 64) & (sb < (c + chunk) // 64))[0]:
+            off = int(sb[i]) * 64 - c
+            sv[i] = xc[off:off + 64]
+        del xc
+    q = lib.quantize(x)
+    assert lib.get_status() == 0
+    e, s2, mu = O.double_quantize(c1)
+    assert q.offset.cpu().numpy().view(np.uint32)[0] == np.float32(mu).view(np.uint32), "mean"
+    assert np.array_equal(q.scale2.cpu().numpy().view(np.uint32), s2.view(np.uint32)), "group scales"
+    assert np.array_equal(q.absmax_e4m3.cpu().numpy(), e), "E4M3 constants"
+    levels, T = O.nf4_codebook()
+    ref_codes = O.nf4_codes(sv.reshape(-1), c1[sb], T).reshape(sb.size, 64)
+    byte_idx = torch.from_numpy((sb[:, None] * 32 + np.arange(32)[None, :]).reshape(-1)).to(dev)
+    got = q.codes[byte_idx].cpu().numpy().reshape(sb.size, 32)
+    assert np.array_equal(got, O.pack_codes(ref_codes.reshape(-1)).reshape(sb.size, 32)), "codes"
+    del x
+    deq = lib.dequantize(q, torch.bfloat16).view(-1)
+    elem_idx = torch.from_numpy((sb[:, None] * 64 + np.arange(64)[None, :]).reshape(-1)).to(dev)
+    got16 = deq[elem_idx].cpu().view(torch.int16).numpy().view(np.uint16).reshape(sb.size, 64)
+    chat = O.fma32(O.e4m3_decode(e[sb]).astype(np.float32), s2[sb // 256], np.float32(mu))
+    ref16 = O.bf16_rne_bits(O.rn32_mul(levels[ref_codes], np.repeat(chat, 64).reshape(sb.size, 64)))
+    assert np.array_equal(got16, ref16), "dequantized bf16"
