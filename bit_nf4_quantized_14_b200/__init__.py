@@ -84,6 +84,8 @@ def _open() -> ctypes.CDLL:
         "qlora_linear_bwd": [vp, vp, i64, P(_NF4Struct), vp, vp, i32, ctypes.c_float, vp, vp, vp, vp,
                              vp, sz, vp],
         "qlora_get_status": [P(i32), vp],
+        "qlora_set_wait_limit": [ctypes.c_uint64],
+        "qlora_selftest_wait": [i32, vp],
         "qlora_error_string": [i32],
         "qlora_profile_enable": [i32],
         "qlora_profile_read": [P(i64), P(ctypes.c_double)],
@@ -448,6 +450,20 @@ def get_status(stream=None) -> int:
     if rc not in (0, -6, -7):
         _check(rc, "qlora_get_status")
     return v.value
+
+
+SELFTEST_MBARRIER, SELFTEST_DEVICE_WORD = 0, 1
+
+
+def set_wait_limit(ns: int) -> None:
+    """qlora_set_wait_limit: how long the kernels' bounded waits last on the current device (0: the
+    default of 2 s). For tests of the timeout path."""
+    _check(load().qlora_set_wait_limit(int(ns)), "qlora_set_wait_limit")
+
+
+def selftest_wait(kind: int, stream=None) -> None:
+    """qlora_selftest_wait: a kernel whose bounded wait must give up (see get_status)."""
+    _check(load().qlora_selftest_wait(int(kind), _stream(stream)), "qlora_selftest_wait")
 
 
 def kernel_launches() -> int:

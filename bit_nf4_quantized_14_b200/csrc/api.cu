@@ -12,6 +12,7 @@
 #include <atomic>
 #include <cstring>
 #include <mutex>
+#include <string>
 #include <vector>
 
 #include "qlora_nf4.h"
@@ -21,6 +22,7 @@
 #include "gemm_nf4w.cuh"
 #include "gemm_sm100.cuh"
 #include "gemv_nf4.cuh"
+#include "selftest.cuh"
 
 namespace qnf4 {
 void build_nf4_codebook(float levels[16], float thresholds[15]);   // codebook.cpp
@@ -46,6 +48,42 @@ inline int launched_at(int line) {
   return e == cudaSuccess ? QLORA_OK : cuda_fail(e, "kernel launch", line);
 }
 #define launched() launched_at(__LINE__)
+
+// Host-side fault injection for tests of callers' error handling: with QLORA_FAULT_INJECT set to
+// "<entry point>" or "<entry point>:<k>", the k-th call (the first by default) of that entry point made
+// since the variable took its current value fails with QLORA_ERR_CUDA, as a launch failure would: after
+// its argument checks, before it enqueues anything. No GPU state is touched.
+std::mutex g_inject_mu;
+std::string g_inject_armed;          // the variable's value when last seen (empty: unset)
+long g_inject_calls = 0;
+std::atomic<bool> g_inject_seen{false};
+bool injected_fault(const char* entry) {
+  const char* v = std::getenv("QLORA_FAULT_INJECT");
+  if (!v || !*v) {
+    if (g_inject_seen.load(std::memory_order_relaxed)) {      // unset since: forget the count
+      std::lock_guard<std::mutex> g(g_inject_mu);
+      g_inject_armed.clear();
+      g_inject_seen.store(false, std::memory_order_relaxed);
+    }
+    return false;
+  }
+  std::lock_guard<std::mutex> g(g_inject_mu);
+  g_inject_seen.store(true, std::memory_order_relaxed);
+  std::string& armed = g_inject_armed;
+  long& calls = g_inject_calls;
+  if (armed != v) { armed = v; calls = 0; }
+  const std::string spec(v);
+  const size_t colon = spec.find(':');
+  const std::string name = spec.substr(0, colon);
+  long k = 1;
+  if (colon != std::string::npos) k = std::strtol(spec.c_str() + colon + 1, nullptr, 10);
+  if (name != entry) return false;
+  if (++calls != k) return false;
+  if (debug_on()) std::fprintf(stderr, "qlora: injected launch failure in %s (call %ld)\n", entry, calls);
+  return true;
+}
+#define INJECT(entry) \
+  do { if (injected_fault(entry)) return QLORA_ERR_CUDA; } while (0)
 
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -572,25 +610,56 @@ constexpr size_t kNoallocSsumBytes = static_cast<size_t>(kNoallocSlabs) * 8;
 static_assert(kNoallocC1Bytes + kNoallocSsumBytes + 256 + 256 == QLORA_NOALLOC_SCRATCH_BYTES, "scratch layout");
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_dev_ptr[kMaxDevices] = {};
+struct NoallocSlot { unsigned long long ctx_id; void* ptr; };
+NoallocSlot g_noalloc_slot[kMaxDevices] = {};
 
 }  // namespace
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[QLORA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-// Device address of this device's scratch array (set-up on the first call per device).
+// Identity of the calling thread's current context: cuCtxGetId through the runtime's driver entry
+// point (the library links no driver library); 0 if it is unavailable.
+unsigned long long current_ctx_id() {
+  using GetCur = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCur get_cur = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<GetCur>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(p);
+  });
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (get_cur && get_cur(&c) == CUDA_SUCCESS && c && get_id && get_id(c, &id) == CUDA_SUCCESS) return id;
+  return 0;
+}
+
+// Device address of this device's scratch array. The set-up -- cudaGetSymbolAddress with the device
+// current -- runs on the first call on a device, and again if that device's context was replaced since
+// (after a cudaDeviceReset the module, and with it the array, may be loaded at another address).
 int noalloc_scratch(void** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail(cudaGetLastError(), "cudaGetDevice", __LINE__);
   if (dev < 0 || dev >= kMaxDevices) return QLORA_ERR_UNSUPPORTED;
+  const unsigned long long ctx = current_ctx_id();
   std::lock_guard<std::mutex> g(g_noalloc_mu);
-  if (!g_noalloc_dev_ptr[dev]) {
+  NoallocSlot& slot = g_noalloc_slot[dev];
+  if (!slot.ptr || ctx == 0 || slot.ctx_id != ctx) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
-    g_noalloc_dev_ptr[dev] = p;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+      return cuda_fail(cudaGetLastError(), "cudaGetSymbolAddress", __LINE__);
+    slot.ptr = p;
+    slot.ctx_id = ctx;
   }
-  *out = g_noalloc_dev_ptr[dev];
+  *out = slot.ptr;
   return QLORA_OK;
 }
 
@@ -704,6 +773,7 @@ int qlora_nf4_quantize(const void* w, int w_dtype, int64_t rows, int64_t cols, c
   if (!aligned16(w) || !aligned16(workspace)) return QLORA_ERR_ALIGNMENT;
   const int64_t n = rows * cols;
   if (!workspace || workspace_bytes < quant_ws(n).total) return QLORA_ERR_WORKSPACE;
+  INJECT("qlora_nf4_quantize");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   ProfScope prof(QLORA_PROF_QUANTIZE, st);
   return run_quantize(w, w_dtype, n, out, workspace, st);
@@ -718,10 +788,13 @@ int qlora_nf4_quantize_noalloc(const void* w, int w_dtype, int64_t rows, int64_t
   if (int e = check_nf4(out)) return e;
   if (out->rows != rows || out->cols != cols) return QLORA_ERR_SHAPE;
   if (!aligned16(w)) return QLORA_ERR_ALIGNMENT;
+  INJECT("qlora_nf4_quantize_noalloc");
   if (int e = check_device(nullptr)) return e;
   void* scratch = nullptr;
   if (int e = noalloc_scratch(&scratch)) return e;
-  return run_quantize(w, w_dtype, rows * cols, out, scratch, reinterpret_cast<cudaStream_t>(stream));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  ProfScope prof(QLORA_PROF_QUANTIZE, st);
+  return run_quantize(w, w_dtype, rows * cols, out, scratch, st);
 }
 
 int qlora_nf4_dequantize(const qlora_nf4_tensor* q, void* out, int out_dtype, qlora_stream_t stream) {
@@ -729,6 +802,7 @@ int qlora_nf4_dequantize(const qlora_nf4_tensor* q, void* out, int out_dtype, ql
   if (out_dtype != QLORA_F32 && out_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
   if (int e = check_nf4(q)) return e;
   if (!aligned16(out)) return QLORA_ERR_ALIGNMENT;
+  INJECT("qlora_nf4_dequantize");
   int sms = 0;
   if (int e = check_device(&sms)) return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -744,6 +818,7 @@ int qlora_nf4_quantize_single(const void* w, int w_dtype, int64_t rows, int64_t 
   if (w_dtype != QLORA_F32 && w_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
   if (rows <= 0 || cols <= 0 || rows > kMaxNumel / cols) return QLORA_ERR_SHAPE;
   if (!aligned16(w) || !aligned16(codes) || !aligned16(absmax)) return QLORA_ERR_ALIGNMENT;
+  INJECT("qlora_nf4_quantize_single");
   int sms = 0;
   if (int e = check_device(&sms)) return e;
   const Buckets& bk = buckets();
@@ -760,6 +835,7 @@ int qlora_nf4_dequantize_single(const void* codes, const float* absmax, int64_t 
   if (out_dtype != QLORA_F32 && out_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
   if (rows <= 0 || cols <= 0 || rows > kMaxNumel / cols) return QLORA_ERR_SHAPE;
   if (!aligned16(codes) || !aligned16(absmax) || !aligned16(out)) return QLORA_ERR_ALIGNMENT;
+  INJECT("qlora_nf4_dequantize_single");
   int sms = 0;
   if (int e = check_device(&sms)) return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -777,6 +853,7 @@ int qlora_codebook_quantize(const void* w, int w_dtype, int64_t n, const float* 
   BucketArg bk;
   if (!make_codebook(levels, nlevels, &cb, &bk)) return QLORA_ERR_CODEBOOK;
   if (!aligned16(w) || !aligned16(codes) || !aligned16(absmax)) return QLORA_ERR_ALIGNMENT;
+  INJECT("qlora_codebook_quantize");
   int sms = 0;
   if (int e = check_device(&sms)) return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -793,6 +870,7 @@ int qlora_codebook_dequantize(const void* codes, const float* absmax, int64_t n,
   BucketArg bk;
   if (!make_codebook(levels, nlevels, &cb, &bk)) return QLORA_ERR_CODEBOOK;
   if (!aligned16(codes) || !aligned16(absmax) || !aligned16(out)) return QLORA_ERR_ALIGNMENT;
+  INJECT("qlora_codebook_dequantize");
   int sms = 0;
   if (int e = check_device(&sms)) return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -821,6 +899,7 @@ int qlora_codebook_stats(const void* w, int w_dtype, const void* codes, const fl
   if (!workspace || workspace_bytes < static_cast<size_t>(G) * kStatVals * sizeof(double)) return QLORA_ERR_WORKSPACE;
   if (!aligned16(w) || !aligned16(codes) || !aligned16(absmax) || !aligned16(stats) || !aligned16(workspace))
     return QLORA_ERR_ALIGNMENT;
+  INJECT("qlora_codebook_stats");
   if (int e = check_device(nullptr)) return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   double* part = static_cast<double*>(workspace);
@@ -845,6 +924,7 @@ int qlora_adamw_step(float* p, const float* g, float* m, float* v, void* p_bf16,
     return QLORA_ERR_INVALID_ARG;
   if (n <= 0 || n > kMaxNumel) return QLORA_ERR_SHAPE;
   if (!aligned16(p) || !aligned16(g) || !aligned16(m) || !aligned16(v) || !aligned16(p_bf16)) return QLORA_ERR_ALIGNMENT;
+  INJECT("qlora_adamw_step");
   int sms = 0;
   if (int e = check_device(&sms)) return e;
   AdamWArgs a;
@@ -912,6 +992,7 @@ int qlora_linear_fwd(const void* X, int64_t T, const qlora_nf4_tensor* W, const 
   if (!Y) return QLORA_ERR_INVALID_ARG;
   if (int e = check_linear(X, T, W, A, B, r, alpha, workspace, workspace_bytes)) return e;
   if (!aligned16(Y) || !aligned16(U_out)) return QLORA_ERR_ALIGNMENT;
+  INJECT("qlora_linear_fwd");
   if (int e = check_device(nullptr)) return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t N = W->rows, K = W->cols;
@@ -946,6 +1027,7 @@ int qlora_linear_bwd(const void* dY, const void* X, int64_t T, const qlora_nf4_t
   if (int e = check_linear(X, T, W, A, B, r, alpha, workspace, workspace_bytes)) return e;
   if (!aligned16(dY) || !aligned16(U) || !aligned16(dX) || !aligned16(dA) || !aligned16(dB))
     return QLORA_ERR_ALIGNMENT;
+  INJECT("qlora_linear_bwd");
   if (int e = check_device(nullptr)) return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t N = W->rows, K = W->cols;
@@ -992,6 +1074,22 @@ int qlora_linear_bwd(const void* dY, const void* X, int64_t T, const qlora_nf4_t
     if (int e = reduce_after(part, N, T, r, bn, 1.0f, dB, Red::kRowsF32, st)) return e;
   }
   return QLORA_OK;
+}
+
+int qlora_set_wait_limit(uint64_t ns) {
+  if (ns != 0 && (ns < 1000 || ns > kWaitLimitNs)) return QLORA_ERR_INVALID_ARG;
+  if (int e = check_device(nullptr)) return e;
+  const unsigned long long v = ns ? ns : kWaitLimitNs;
+  if (cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)) != cudaSuccess)
+    return cuda_fail(cudaGetLastError(), "cudaMemcpyToSymbol", __LINE__);
+  return QLORA_OK;
+}
+
+int qlora_selftest_wait(int kind, qlora_stream_t stream) {
+  if (kind != QLORA_SELFTEST_MBARRIER && kind != QLORA_SELFTEST_DEVICE_WORD) return QLORA_ERR_INVALID_ARG;
+  if (int e = check_device(nullptr)) return e;
+  bounded_wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(kind);
+  return launched();
 }
 
 int qlora_get_status(int* device_status, qlora_stream_t stream) {

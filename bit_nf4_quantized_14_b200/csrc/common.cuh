@@ -20,8 +20,10 @@ __device__ unsigned int g_status;
 __device__ __forceinline__ void raise_status(unsigned bits) { atomicOr(&g_status, bits); }
 
 // A bounded wait gives up after this many nanoseconds of device time and reports a timeout; no
-// legitimate wait in these kernels comes within orders of magnitude of it.
+// legitimate wait in these kernels comes within orders of magnitude of it. The limit in force is the
+// per-device word g_wait_limit_ns (qlora_set_wait_limit shortens it for tests of the timeout path).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+__device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;
@@ -62,13 +64,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait for the phase with the given parity to complete. Returns false (and records a timeout in the
-// status word) if it has not completed within kWaitLimitNs.
+// status word) if it has not completed within the wait limit in force (g_wait_limit_ns).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
+  const unsigned long long t0 = globaltimer_ns(), limit = *(volatile unsigned long long*)&g_wait_limit_ns;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit) {
+      raise_status(kStatusTimeout);
+      return false;
+    }
+  }
+}
+// Wait until the 64-bit word at p (global memory, written by another CTA of the same grid) equals
+// `want`, with acquire ordering for what its writer published before it. Bounded like mbar_wait.
+__device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u64(uint64_t* p, uint64_t v) {
+  asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ bool wait_word_eq(const uint64_t* p, uint64_t want) {
+  if (ld_acquire_u64(p) == want) return true;
+  const unsigned long long t0 = globaltimer_ns(), limit = *(volatile unsigned long long*)&g_wait_limit_ns;
+  while (true) {
+    __nanosleep(64);
+    if (ld_acquire_u64(p) == want) return true;
+    if (globaltimer_ns() - t0 > limit) {
       raise_status(kStatusTimeout);
       return false;
     }

@@ -286,6 +286,33 @@ int qlora_linear_bwd(const void* dY, const void* X, int64_t T, const qlora_nf4_t
  */
 int qlora_get_status(int* device_status, qlora_stream_t stream);
 
+/*
+ * Failure-path controls for tests (the pages have no counterpart; the bounded waits and the status word
+ * are this library's own error handling).
+ *
+ * qlora_set_wait_limit sets, for the current device, how long (ns, device time) any bounded wait in the
+ * library's kernels -- on a shared-memory barrier, or on a device word written by another CTA of the
+ * same grid -- waits before it gives up, records QLORA_STATUS_TIMEOUT and lets its kernel unwind. 0
+ * restores the default of 2 s; other values must lie in [1000, 2e9]. Every later launch on the device
+ * uses the new limit, so a short limit can make long legitimate waits fail: it is meant for tests.
+ * Synchronous (a copy to device memory). QLORA_ERR_INVALID_ARG for a value out of range.
+ *
+ * qlora_selftest_wait launches, on `stream`, a one-warp kernel that waits on something that never
+ * happens: kind QLORA_SELFTEST_MBARRIER waits on a shared-memory barrier that no thread arrives on,
+ * QLORA_SELFTEST_DEVICE_WORD on a device word that nothing writes. The wait gives up after the limit in
+ * force and the kernel returns; qlora_get_status then reports QLORA_ERR_TIMEOUT and the context stays
+ * usable. Nothing faults, traps or spins without a bound.
+ *
+ * Host-side fault injection: with the environment variable QLORA_FAULT_INJECT set to "<entry point>"
+ * or "<entry point>:<k>" (e.g. "qlora_linear_fwd:2"), the k-th call (default: the first) of that entry
+ * point since the variable took its current value returns QLORA_ERR_CUDA, as a failed launch would,
+ * after its argument checks and before it enqueues anything. With QLORA_DEBUG set, each injected failure
+ * is reported on stderr. Applies to the entry points that launch kernels.
+ */
+enum { QLORA_SELFTEST_MBARRIER = 0, QLORA_SELFTEST_DEVICE_WORD = 1 };
+int qlora_set_wait_limit(uint64_t ns);
+int qlora_selftest_wait(int kind, qlora_stream_t stream);
+
 /* Static English text for a QLORA_* code (never NULL). */
 const char* qlora_error_string(int code);
 

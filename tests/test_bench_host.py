@@ -30,6 +30,20 @@ def test_roofline_picks_the_dominant_class():
     assert bench.roofline(prof, 1, peaks, "measured")["bound"] == "hbm"
 
 
+def test_roofline_peak_burst_for_a_short_region_at_full_clock():
+    prof = {"quantize": (3, 0.5), "dequantize": (3, 0.2), "fwd_gemm": (3, 3.6), "bwd_gemm": (3, 3.5), "lora": (30, 0.4)}
+    peaks = {"hbm_gbs": 6543.1, "bf16_tflops": 1636.3, "bf16_tflops_sustained": 1375.0}
+    full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965}
+    rf = bench.roofline(prof, 1, peaks, "measured", timed_s=0.09, clk=full)
+    assert rf["peak"] == 1636.3 and "burst" in rf["peak_source"]
+    assert abs(rf["frac"] - rf["achieved"] / 1636.3) < 1e-3
+    # a long region, or a clock held below its maximum, keeps the sustained figure
+    assert bench.roofline(prof, 1, peaks, "measured", timed_s=4.0, clk=full)["peak"] == 1375.0
+    low = {"sm_mhz": 1312.0, "sm_max_mhz": 1965}
+    assert bench.roofline(prof, 1, peaks, "measured", timed_s=0.09, clk=low)["peak"] == 1375.0
+    assert bench.roofline(prof, 1, peaks, "measured", timed_s=0.09, clk=None)["peak"] == 1375.0
+
+
 def _worker(rank, world, port, q):
     import torch.distributed as dist
     os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))

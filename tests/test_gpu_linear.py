@@ -138,8 +138,8 @@ def test_persistent_tiles_full_compare(lib, N, K):
 @pytest.mark.parametrize("T", [1, 2, 4, 7, 8, 9, 16, 17, 32, 33, 64])
 @pytest.mark.parametrize("N,K,r", [(520, 704, 24), (1000, 320, 64)])
 def test_small_token_forward(lib, T, N, K, r):
-    """T <= 64 runs the GEMV kernels: tails in rows (240-row tiles), in the contraction (256-wide stages),
-    in tokens (8-wide MMA tiles) and in r (16-deep MMA steps). Y and U against the oracle; the backward
+    """T <= 64 runs the small-token kernels: tails in rows (partial row tiles), in the contraction
+    (partial stages), in tokens (8-wide MMA tiles) and in r (16-deep MMA steps). Y and U against the oracle; the backward
     (GEMM path) against the oracle as well, with U from this forward and recomputed."""
     case = synth.linear_case(T=T, N=N, K=K, r=r, alpha=16.0, seed=11 + T)
     errs, (Y, U, dX, dA, dB), q, d = run_and_check(lib, case)
@@ -175,10 +175,13 @@ def test_gemv_and_gemm_paths_at_the_boundary(lib, T):
     run_and_check(lib, case)
 
 
-@pytest.mark.parametrize("N,K,Ts", [(8192, 8192, (1, 4, 16)), (4096, 11008, (16,))])
+@pytest.mark.parametrize("N,K,Ts", [(8192, 8192, (1, 4, 16)), (22016, 8192, (1, 4, 16)), (8192, 22016, (1, 4, 16)),
+                                    (4096, 11008, (16,))])
 def test_decode_shapes(lib, N, K, Ts):
-    """The decode-shaped layers (65B-sized 8192 x 8192; the wide contraction of a down projection) at the
-    decode token counts: every output of Y and U against the oracle (fp64 GEMM over the exact W_hat)."""
+    """The decode-shaped layers of a 65B model (attention 8192 x 8192, gate/up 22016 x 8192, down
+    8192 x 22016) at the decode token counts, plus the wide contraction of a 7B down projection: every
+    output of Y and U against the oracle (fp64 GEMM over the oracle's exact W_hat). The 22016-row and
+    22016-deep layers are the ones whose row and contraction counts leave partial tiles and stages."""
     case = synth.linear_case(T=max(Ts), N=N, K=K, r=64, alpha=16.0, seed=25)
     q, Wt, d, h = setup(lib, case)
     for T in Ts:
@@ -188,3 +191,15 @@ def test_decode_shapes(lib, N, K, Ts):
         Yr, Ur = O.linear_fwd(h["X"][:T], Wt, h["A"], h["B"], 16.0)
         assert rel(Y.float().cpu(), Yr) <= TOL, T
         assert rel(U.float().cpu(), (16.0 / 64) * Ur) <= TOL, T
+
+
+def test_small_token_and_gemm_paths_agree(lib):
+    """The same 64 tokens through the small-token path (T = 64) and, as the first 64 of 65 tokens,
+    through the fused GEMM path: the two results agree with each other within the oracle tolerance."""
+    case = synth.linear_case(T=65, N=2048, K=1536, r=64, alpha=16.0, seed=26)
+    q, Wt, d, h = setup(lib, case)
+    Y64, U64 = lib.linear_fwd(d["X"][:64].contiguous(), q, d["A"], d["B"], 16.0)
+    Y65, U65 = lib.linear_fwd(d["X"], q, d["A"], d["B"], 16.0)
+    assert lib.get_status() == 0
+    assert rel(Y64.float().cpu(), Y65[:64].float().cpu()) <= TOL
+    assert rel(U64.float().cpu(), U65[:64].float().cpu()) <= TOL

@@ -215,3 +215,34 @@ def test_codebook_density_rule(q):
         assert L.qlora_codebook_quantize(W, 0, 4096, arr, 3, C, A, None) == -10, lv
         rejected += 1
     assert rejected == 19
+
+
+def test_fault_injection_fails_the_chosen_call_on_the_host():
+    """QLORA_FAULT_INJECT=<entry>:<k> fails exactly the k-th call of that entry point, after its argument
+    checks (a call with a bad argument is not counted) and before any CUDA call; QLORA_DEBUG reports it.
+    Run in a child process so the variables apply from the library's first call."""
+    import subprocess
+    import sys
+    code = r"""
+import ctypes, sys
+sys.path.insert(0, ROOT)
+import bit_nf4_quantized_14_b200 as q
+L = q.lib
+st = q._NF4Struct(0x100000, 0x110000, 0x120000, 0x130000, 4, 64)
+V = ctypes.c_void_p
+call = lambda w: L.qlora_nf4_quantize(V(w), 0, 4, 64, ctypes.byref(st), V(0x200000), 1 << 20, None)
+print("RC", call(0x300008), call(0x300000), call(0x300000), call(0x300000), flush=True)
+print("WL", L.qlora_set_wait_limit(10), L.qlora_set_wait_limit(1 << 40), L.qlora_selftest_wait(9, None), flush=True)
+"""
+    env = dict(os.environ, QLORA_FAULT_INJECT="qlora_nf4_quantize:2", QLORA_DEBUG="1", CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, "-c", f"ROOT = {ROOT!r}\n" + code], capture_output=True, text=True,
+                       env=env, timeout=300)
+    assert r.returncode == 0, r.stderr
+    rc = [int(v) for v in next(l for l in r.stdout.splitlines() if l.startswith("RC")).split()[1:]]
+    assert rc[0] == -3                       # misaligned: rejected before the injection point, not counted
+    assert rc[1] in (-5, -8) and rc[3] in (-5, -8)   # no GPU in the child: the device check fails
+    assert rc[2] == -5
+    injected = [l for l in r.stderr.splitlines() if "injected launch failure" in l]
+    assert injected == ["qlora: injected launch failure in qlora_nf4_quantize (call 2)"]
+    wl = [int(v) for v in next(l for l in r.stdout.splitlines() if l.startswith("WL")).split()[1:]]
+    assert wl == [-1, -1, -1]

@@ -52,6 +52,26 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls(lib):
     _same(got, lib.quantize(wb))
 
 
+def test_noalloc_back_to_back_on_one_stream(lib):
+    """Stream order is what makes the shared scratch safe: two calls enqueued one after the other on one
+    non-default stream, with no synchronization between them, each equal the workspace entry point's
+    result bit for bit."""
+    W1 = torch.from_numpy(synth.weight_f32(2048, 3072, seed=0, tensor_id=64)).cuda()
+    W2 = torch.from_numpy(synth.sweep_f32(5 * 16384 + 4097, seed=0, tensor_id=65).reshape(1, -1)).cuda()
+    refs = [lib.quantize(W1), lib.quantize(W2)]
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    outs = [lib.NF4Weight.empty(w.shape[0], w.shape[1], w.device) for w in (W1, W2)]
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for w, o in zip((W1, W2), outs):
+            assert _noalloc(lib, w, o) == 0
+    side.synchronize()
+    assert lib.get_status(side) == 0
+    for o, ref in zip(outs, refs):
+        _same(o, ref)
+
+
 def test_noalloc_rejects_inputs_beyond_its_scratch(lib):
     n = lib.NOALLOC_MAX_NUMEL
     fake = lib.NF4Weight.empty(1, 64, "cuda")
