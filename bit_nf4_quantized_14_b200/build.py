@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libqlora_nf4.so")
 SOURCES = [os.path.join(HERE, "csrc", f) for f in ("api.cu", "codebook.cpp")]
 HEADERS = [os.path.join(HERE, "csrc", f) for f in ("common.cuh", "codec.cuh", "codebook_study.cuh", "gemm_sm100.cuh", "gemm_nf4w.cuh",
-                                                              "gemv_nf4.cuh", "adamw.cuh", "selftest.cuh")] + [
+                                                              "gemv_nf4.cuh", "adamw.cuh", "selftest.cuh", "decode_nf4.cuh")] + [
     os.path.join(ROOT, "include", "qlora_nf4.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",

@@ -12,6 +12,7 @@
 #include <atomic>
 #include <cstring>
 #include <mutex>
+#include <random>
 #include <string>
 #include <vector>
 
@@ -22,6 +23,7 @@
 #include "gemm_nf4w.cuh"
 #include "gemm_sm100.cuh"
 #include "gemv_nf4.cuh"
+#include "decode_nf4.cuh"
 #include "selftest.cuh"
 
 namespace qnf4 {
@@ -263,6 +265,27 @@ bool make_tmap_t(CUtensorMap* m, const void* ptr, TmType t, uint64_t inner, uint
                  box_inner, box_outer, (int)swizzle128, (int)r);
   return r == CUDA_SUCCESS;
 }
+// 3-D tensor: dims[0] contiguous elements, dims[1] and dims[2] with byte strides strides[0], strides[1].
+bool make_tmap_3d(CUtensorMap* m, const void* ptr, TmType t, const uint64_t (&dims)[3], const uint64_t (&strides)[2],
+                  const uint32_t (&box)[3], bool swizzle128) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const CUtensorMapDataType dt = t == TmType::kBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                 : t == TmType::kU8  ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+  cuuint64_t st[2] = {strides[0], strides[1]};
+  cuuint32_t bx[3] = {box[0], box[1], box[2]};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, dt, 3, const_cast<void*>(ptr), d, st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS && debug_on())
+    std::fprintf(stderr, "qlora: 3-D tensor map (ptr %p, dims %llu x %llu x %llu, box %u x %u x %u) -> %d\n", ptr,
+                 (unsigned long long)dims[0], (unsigned long long)dims[1], (unsigned long long)dims[2], box[0], box[1],
+                 box[2], (int)r);
+  return r == CUDA_SUCCESS;
+}
 bool make_tmap(CUtensorMap* m, const void* ptr, bool bf16, uint64_t inner, uint64_t outer,
                uint32_t box_inner, uint32_t box_outer, bool swizzle128 = true) {
   return make_tmap_t(m, ptr, bf16 ? TmType::kBf16 : TmType::kU8, inner, outer, inner, box_inner, box_outer,
@@ -471,10 +494,34 @@ GemvWs gemv_ws(int64_t T, int64_t N, int64_t K, int r) {
   return w;
 }
 
+// ---- decode path (T <= kDcMaxTokens): one cooperative launch of nf4_decode_kernel ---------------
+// Workspace of the decode path (offsets in bytes): one tag per 8-row unit of A, and the per-CTA results
+// awaiting the adapter term when they do not fit in shared memory.
+struct DecWs { size_t tags, base, total; };
+DecWs dec_ws(int64_t T, int64_t N, int r) {
+  DecWs w;
+  w.tags = 0;
+  w.base = align256(static_cast<size_t>(r / 8) * 8);
+  w.total = w.base + align256(static_cast<size_t>(T) * N * 4);
+  return w;
+}
+// A value no earlier call in this process used and that uninitialised memory is unlikely to hold: the
+// tree's tags compare equal to it only once this call has written them.
+uint64_t next_call_tag() {
+  static std::atomic<uint64_t> ctr{[] {
+    std::random_device rd;
+    return (static_cast<uint64_t>(rd()) << 32) ^ rd() ^ 0x9E3779B97F4A7C15ull;
+  }()};
+  uint64_t v;
+  do { v = ctr.fetch_add(1, std::memory_order_relaxed); } while (v == 0 || v == ~0ull);
+  return v;
+}
+
 LinearWs linear_ws(int64_t T, int64_t N, int64_t K, int r) {
   const int bn = static_cast<int>(cdiv(r, 64) * 64);
   int64_t part = 0;
   if (T <= kGvMaxTokens) part = static_cast<int64_t>(gemv_ws(T, N, K, r).total / 4);
+  if (T <= kDcMaxTokens) part = std::max<int64_t>(part, static_cast<int64_t>(dec_ws(T, N, r).total / 4));
   part = std::max(part, skinny_part_elems(T, K, bn));   // U
   part = std::max(part, skinny_part_elems(T, N, bn));   // V
   part = std::max(part, skinny_part_elems(K, T, bn));   // dA
@@ -586,6 +633,68 @@ int gemv_fwd(const void* X, int64_t T, const qlora_nf4_tensor* W, const void* B,
     case 4: return launch_gemv_nt<4>(ta, tx, p, G, st);
     default: return launch_gemv_nt<8>(ta, tx, p, G, st);
   }
+}
+
+// Decode-sized forward (or, with u_only, the adapter projection sU alone) in one cooperative launch:
+// one CTA per SM, every CTA resident, which the waits for sU written by other CTAs require. sU's
+// summation order does not depend on the grid, so the backward's recompute gives the forward's U.
+int launch_decode(const void* X, int64_t T, const qlora_nf4_tensor* W, const void* A, const void* B, int r, float s,
+                  void* Y, void* U, char* dws, bool u_only, cudaStream_t st) {
+  int sms = 0;
+  if (int e = check_device(&sms)) return e;
+  const int64_t N = W->rows, K = W->cols;
+  const DecWs L = dec_ws(T, N, r);
+  const int64_t units = N / 8, aunits = r / 8;
+  const int G = static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>(units + kDcALoad * aunits, std::min(sms, kGvMaxCtas))));
+  // codes as (32 bytes of a block, row, block); A as (64 elements of a block, row, block); one box height per
+  // pass size
+  const uint64_t nkb = static_cast<uint64_t>(K / 64);
+  DcMaps maps;
+  bool ok = make_tmap_t(&maps.b, B, TmType::kBf16, r, N, r, std::min(r, 64), 8, false);
+  for (int h = 1; ok && h <= kDcUnits; ++h)
+    ok = make_tmap_3d(&maps.c[h - 1], W->codes, TmType::kU8, {32, static_cast<uint64_t>(N), nkb},
+                      {static_cast<uint64_t>(K / 2), 32}, {32, static_cast<uint32_t>(8 * h), kDcStageBlocks}, false);
+  for (int h = 1; ok && h <= kDcAUnits; ++h)
+    ok = make_tmap_3d(&maps.a[h - 1], A, TmType::kBf16, {64, static_cast<uint64_t>(r), nkb},
+                      {static_cast<uint64_t>(K) * 2, 128}, {64, static_cast<uint32_t>(8 * h), kDcStageBlocks}, true);
+  if (!ok) return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
+  DecParams p{};
+  p.T = static_cast<int>(T); p.N = static_cast<int>(N); p.K = static_cast<int>(K); p.r = r;
+  p.RP = static_cast<int>(cdiv(r, 64) * 64);
+  p.nkb = static_cast<int>(K / 64);
+  p.units = static_cast<int>(units);
+  p.aunits = static_cast<int>(aunits);
+  p.u_only = u_only ? 1 : 0;
+  // the most NF4 units one CTA can get (see dc_share): ceil(L / G) load positions
+  const int64_t per_cta = cdiv(units + kDcALoad * aunits, G);
+  p.base_in_smem = per_cta * T * 8 * 4 <= kDcBaseBytes ? 1 : 0;
+  p.s = s;
+  p.X = static_cast<const __nv_bfloat16*>(X);
+  p.e4m3 = W->absmax_e4m3;
+  p.s2 = W->scale2;
+  p.mu = W->offset;
+  p.Y = static_cast<__nv_bfloat16*>(Y);
+  p.U = static_cast<__nv_bfloat16*>(U);
+  p.tags = reinterpret_cast<uint64_t*>(dws + L.tags);
+  p.base_ws = reinterpret_cast<float*>(dws + L.base);
+  p.seq = next_call_tag();
+  auto kern = T <= 8 ? nf4_decode_kernel<8> : nf4_decode_kernel<16>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDcSmemBytes) != cudaSuccess)
+    return cuda_fail(cudaGetLastError(), "cudaFuncSetAttribute", __LINE__);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(G));
+  cfg.blockDim = dim3(kDcThreads);
+  cfg.dynamicSmemBytes = kDcSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, maps, p, codebook()) != cudaSuccess)
+    return cuda_fail(cudaGetLastError(), "cooperative launch", __LINE__);
+  return launched();
 }
 
 int compute_sU(const void* X, int64_t T, int64_t K, const void* A, int r, float s, void* sU, float* part,
@@ -1001,7 +1110,11 @@ int qlora_linear_fwd(const void* X, int64_t T, const qlora_nf4_tensor* W, const 
   char* ws = static_cast<char*>(workspace);
   void* sU = U_out ? U_out : ws + L.sU;
   float* part = reinterpret_cast<float*>(ws + L.part);
-  if (T <= kGvMaxTokens) {                      // decode-sized: the stream-K GEMV kernels
+  if (T <= kDcMaxTokens) {                      // decode-sized: one launch, projection included
+    ProfScope prof(QLORA_PROF_FWD_GEMM, st);
+    return launch_decode(X, T, W, A, B, r, s, Y, sU, ws + L.part, false, st);
+  }
+  if (T <= kGvMaxTokens) {                      // small token counts: the stream-K GEMV kernels
     int sms = 0;
     if (int e = check_device(&sms)) return e;
     const GemvWs G = gemv_ws(T, N, K, r);
@@ -1041,7 +1154,9 @@ int qlora_linear_bwd(const void* dY, const void* X, int64_t T, const qlora_nf4_t
   {
     ProfScope prof(QLORA_PROF_LORA, st);
     if (!sU) {                                  // the forward's own projection, so U is identical
-      if (T <= kGvMaxTokens) {
+      if (T <= kDcMaxTokens) {
+        if (int e = launch_decode(X, T, W, A, B, r, s, nullptr, ws + L.sU, ws + L.part, true, st)) return e;
+      } else if (T <= kGvMaxTokens) {
         if (int e = gemv_sU(X, T, K, A, r, s, ws + L.sU, ws + L.part, gemv_ws(T, N, K, r), st)) return e;
       } else if (int e = compute_sU(X, T, K, A, r, s, ws + L.sU, part, st)) {
         return e;

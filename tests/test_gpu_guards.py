@@ -57,7 +57,8 @@ def test_codec_outputs_stay_inside_their_buffers(lib, n, dtype):
         o = Guarded(n, out_dtype)
         lib.dequantize(q, out_dtype, out=o.t.reshape(1, n))
         assert o.intact(), tag
-        got = o.t.cpu().numpy().view(np.uint16 if tag == "bf16" else np.uint32)
+        got = o.t.cpu().view(torch.int16 if tag == "bf16" else torch.int32).numpy().view(
+            np.uint16 if tag == "bf16" else np.uint32)
         assert np.array_equal(got, O.dequantize(ref, tag).reshape(-1).view(got.dtype)), tag
 
 
@@ -80,6 +81,7 @@ def test_single_and_noalloc_outputs_stay_inside_their_buffers(lib, n):
 
 @pytest.mark.parametrize("T,N,K,r", [(1, 264, 192, 8), (3, 1000, 320, 24), (9, 8, 64, 8), (17, 520, 704, 64),
                                      (33, 136, 1088, 136), (64, 1032, 128, 16), (65, 392, 320, 24),
+                                     (12, 200, 640, 136), (2, 11848, 128, 16),
                                      (129, 520, 128, 64), (300, 8, 576, 256)])
 def test_linear_outputs_stay_inside_their_buffers(lib, T, N, K, r):
     """Both the small-token path (T <= 64) and the fused GEMM path, with tails in every tile dimension."""

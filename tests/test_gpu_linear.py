@@ -203,3 +203,20 @@ def test_small_token_and_gemm_paths_agree(lib):
     assert lib.get_status() == 0
     assert rel(Y64.float().cpu(), Y65[:64].float().cpu()) <= TOL
     assert rel(U64.float().cpu(), U65[:64].float().cpu()) <= TOL
+
+
+@pytest.mark.parametrize("T,N,K,r", [(2, 11848, 128, 16),     # ~10 row units per CTA: two passes
+                                     (16, 45056, 64, 8),      # per-CTA results kept in the workspace
+                                     (12, 200, 640, 136),     # r > 64: several adapter column boxes
+                                     (4, 64, 256, 256),       # the largest rank
+                                     (7, 96, 1088, 64),       # 17 blocks: a last stage with one block
+                                     (16, 8, 64, 8)])         # one row unit: a one-CTA grid
+def test_decode_path_structure(lib, T, N, K, r):
+    """The decode-sized path (T <= 16) in the configurations its structure depends on; Y and U against
+    the oracle, and the backward's recomputed U bit-identical to the forward's."""
+    case = synth.linear_case(T=T, N=N, K=K, r=r, alpha=16.0, seed=27)
+    errs, (Y, U, dX, dA, dB), q, d = run_and_check(lib, case)
+    dX2, dA2, dB2 = lib.linear_bwd(d["dY"], d["X"], q, d["A"], d["B"], 16.0, U=None)
+    assert torch.equal(dA, dA2) and torch.equal(dB, dB2) and torch.equal(dX, dX2)
+    Y2, U2 = lib.linear_fwd(d["X"], q, d["A"], d["B"], 16.0)
+    assert torch.equal(Y, Y2) and torch.equal(U, U2)
