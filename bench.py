@@ -575,8 +575,8 @@ def secondary_figures(q, device, reps=20, warmup=3):
     peaks, kind = load_peaks()
     gen = torch.Generator(device=device)
     gen.manual_seed(2026)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
-    out = {"l2": "flushed (512 MB write) before every timed call; median of %d calls, CUDA events" % reps,
+    flush = L2Flush(device)
+    out = {"l2": L2_NOTE + "; median of %d calls, CUDA events" % reps,
            "peak": peaks["hbm_gbs"], "peak_source": f"{kind} (HBM copy)"}
     N, K, T = SECONDARY_DECODE
     W = device_weight(N, K, gen)
@@ -592,11 +592,15 @@ def secondary_figures(q, device, reps=20, warmup=3):
     q.linear_fwd(X, nf4, A, B, ALPHA, out=Y, U_out=U, workspace=ws)
     launches = q.kernel_launches() - n0
     ms = time_calls(lambda: q.linear_fwd(X, nf4, A, B, ALPHA, out=Y, U_out=U, workspace=ws), flush, reps, warmup)
+    ring = [nf4] + [nf4_copy(q, nf4) for _ in range(CHAIN_WEIGHTS - 1)]
+    ms_chain = time_chain([lambda w=w: q.linear_fwd(X, w, A, B, ALPHA, out=Y, U_out=U, workspace=ws) for w in ring],
+                          CHAIN_CALLS)
     byt = gemv_bytes(T, N, K, RANK_R)
     out["decode"] = {"workload": f"QLoRA linear forward, NF4 W {N} x {K}, T = {T}, r = {RANK_R}", "us": round(ms * 1e3, 2),
                      "bytes": int(byt), "GB/s": round(byt / (ms / 1e3) / 1e9, 1),
-                     "frac": round(byt / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4), "launches_per_call": launches}
-    del nf4, A, B, X, Y, U, ws
+                     "frac": round(byt / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4), "launches_per_call": launches,
+                     "chain": chain_entry(ms_chain, byt, peaks)}
+    del nf4, ring, A, B, X, Y, U, ws
     n = SECONDARY_SWEEP_N
     x = device_sweep(n, gen).view(1, n)
     xb = x.to(torch.bfloat16)
@@ -631,16 +635,57 @@ def gemv_bytes(T, N, K, r):
     return (0.5 + 1 / 64 + 4 / 16384) * N * K + 2 * r * (N + K) + 2 * T * (N + K)
 
 
+CHAIN_WEIGHTS = 6     # distinct copies of the weight a chain cycles through (6 x 34 MB and more: > L2)
+CHAIN_CALLS = 16
+
+
+def nf4_copy(q, w):
+    """A copy of an NF4 weight in new device memory (same values, distinct addresses)."""
+    return q.NF4Weight(w.codes.clone(), w.absmax_e4m3.clone(), w.scale2.clone(), w.offset.clone(), w.rows, w.cols)
+
+
+def chain_entry(ms, byt, peaks):
+    return {"us": round(ms * 1e3, 2), "GB/s": round(byt / (ms / 1e3) / 1e9, 1),
+            "frac": round(byt / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+            "how": f"{CHAIN_CALLS} calls back to back over {CHAIN_WEIGHTS} copies of the weight in distinct memory "
+                   "(consecutive layers of a decode step), enqueued behind a device sleep; no flush"}
+
+
+L2_NOTE = ("flushed before every timed call: a 512 MB write, then a read of another 512 MB buffer, so the "
+           "timed call finds neither its inputs nor dirty lines in L2")
+
+
+class L2Flush:
+    """Evict what the next timed call reads from L2 and leave L2 clean. A 512 MB write (4x the 126 MB L2)
+    evicts everything but leaves L2 full of dirty lines, which the timed call then pays to write back as
+    it evicts them (for a 90 MB read, about a third more time; `--workload flush_check` measures it); a
+    full read of a second 512 MB buffer afterwards replaces them with clean lines of that buffer."""
+
+    def __init__(self, device):
+        import torch
+        self.w = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+        self.r = torch.zeros(64 << 20, dtype=torch.int64, device=device)
+        self.i = 0
+
+    def write_only(self):
+        self.i += 1
+        self.w.fill_(self.i & 0xFF)
+
+    def __call__(self):
+        self.write_only()
+        self.r.sum()
+
+
 def time_calls(fn, flush, reps, warmup=3):
-    """Median device time (ms) of fn() over reps calls, the L2 flushed by a 512 MB write before each
-    (outside the timed pair of events, on the same stream)."""
+    """Median device time (ms) of fn() over reps calls, the L2 flushed (flush()) before each, outside the
+    timed pair of events, on the same stream."""
     import torch
     for _ in range(warmup):
         fn()
     stream = torch.cuda.current_stream()
     times = []
     for i in range(reps):
-        flush.fill_(i & 0xFF)
+        flush()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         fn()
@@ -650,18 +695,64 @@ def time_calls(fn, flush, reps, warmup=3):
     return statistics.median(times)
 
 
+def time_chain(fns, calls, reps=5):
+    """Median per-call device time (ms) of `calls` calls enqueued back to back, cycling through fns (calls on
+    distinct weights whose total exceeds L2, as the layers of a decode step do), behind a 1 ms device sleep
+    so the host's enqueueing is not timed."""
+    import torch
+    for f in fns:
+        f()
+    stream = torch.cuda.current_stream()
+    per = []
+    for _ in range(reps):
+        torch.cuda._sleep(2_000_000)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(calls):
+            fns[i % len(fns)]()
+        b.record(stream)
+        b.synchronize()
+        per.append(a.elapsed_time(b) / calls)
+    return statistics.median(per)
+
+
+def run_flush_check(args):
+    """How the L2 flush before a timed call changes what it measures, on a plain torch read (a sum over
+    90 MB and 34 MB, the sizes of the decode layers' NF4 weights): after a write-only flush, after the
+    write-then-read flush the other measurement lines use, with no flush (inputs L2-resident), and as a
+    chain over distinct copies. Library kernels only; none of this package's."""
+    import torch
+    device = torch.device("cuda", 0)
+    flush = L2Flush(device)
+    cases = []
+    for mb in (90, 34):
+        ring = [torch.ones((mb << 20) // 8, dtype=torch.int64, device=device) for _ in range(CHAIN_WEIGHTS)]
+        fn = lambda: ring[0].sum()
+        row = {"MB": mb}
+        row["write_flush_us"] = round(time_calls(fn, flush.write_only, args.steps, args.warmup) * 1e3, 2)
+        row["write_read_flush_us"] = round(time_calls(fn, flush, args.steps, args.warmup) * 1e3, 2)
+        row["no_flush_us"] = round(time_calls(fn, lambda: None, args.steps, args.warmup) * 1e3, 2)
+        row["chain_us"] = round(time_chain([lambda t=t: t.sum() for t in ring], CHAIN_CALLS) * 1e3, 2)
+        cases.append(row)
+        del ring
+    print(json.dumps({"metric": "device time of a torch sum over a weight-sized tensor under each L2 preparation",
+                      "unit": "us", "steps": args.steps, "warmup": args.warmup, "cases": cases}), flush=True)
+    return 0
+
+
 def run_decode(args):
     import torch
     import synth
     import bit_nf4_quantized_14_b200 as q
     peaks, kind = load_peaks()
     device = torch.device("cuda", 0)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
     cases = []
     for i, (N, K) in enumerate(synth.LLAMA65B_SHAPES):
         W = torch.from_numpy(synth.weight_f32(N, K, seed=40 + i, tensor_id=1)).to(device)
         nf4 = q.quantize(W)
         del W
+        ring = [nf4] + [nf4_copy(q, nf4) for _ in range(CHAIN_WEIGHTS - 1)]
         A = synth.to_bf16(synth.normal_f32((RANK_R, K), 0.01, 40 + i, 3)).to(device)
         B = synth.to_bf16(synth.normal_f32((N, RANK_R), 0.01, 40 + i, 4)).to(device)
         X16 = synth.to_bf16(synth.normal_f32((max(DECODE_TOKENS), K), 1.0, 40 + i, 2)).to(device)
@@ -675,17 +766,21 @@ def run_decode(args):
             fn()
             launches = q.kernel_launches() - n0
             ms = time_calls(fn, flush, args.steps, args.warmup)
+            ms_chain = time_chain([lambda w=w: q.linear_fwd(X, w, A, B, ALPHA, out=Y, U_out=U, workspace=ws)
+                                   for w in ring], CHAIN_CALLS)
             gbs = gemv_bytes(T, N, K, RANK_R) / (ms / 1e3) / 1e9
             cases.append({"N": N, "K": K, "T": T, "us": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
                           "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes": int(gemv_bytes(T, N, K, RANK_R)),
-                          "launches_per_call": launches})
+                          "launches_per_call": launches,
+                          "chain": chain_entry(ms_chain, gemv_bytes(T, N, K, RANK_R), peaks)})
+        del ring
     status = q.get_status()
     gm = math.exp(sum(math.log(c["GB/s"]) for c in cases) / len(cases))
     print(json.dumps({"metric": "QLoRA decode-shaped linear forward, HBM GB/s (geomean over cases)",
                       "value": round(gm, 1), "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
                       "warmup": args.warmup, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
                       "config": {"workload": DECODE_WORKLOAD, "r": RANK_R, "alpha": ALPHA,
-                                 "l2": "flushed (512 MB write) before every timed call"},
+                                 "l2": L2_NOTE},
                       "roofline": {"bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"],
                                    "peak_source": f"{kind} (HBM copy)", "achieved": round(gm, 1),
                                    "frac": round(gm / peaks["hbm_gbs"], 4)},
@@ -699,7 +794,7 @@ def run_codec_sweep(args):
     import bit_nf4_quantized_14_b200 as q
     peaks, kind = load_peaks()
     device = torch.device("cuda", 0)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
     chunk = 1 << 28          # the largest sizes are concatenations of independent 2^28-element sweep tensors
     nmax = max(SWEEP_SIZES)
     x = torch.empty(nmax, dtype=torch.float32, device=device)
@@ -741,7 +836,7 @@ def run_codec_sweep(args):
                       "data": "synthetic",
                       "config": {"workload": "sweep tensors: rows of 4096, sigma_row ~ U(0.005, 0.05), 0.1 % x10 "
                                              "outliers; sizes 2^20..2^30 (2^30 = four 2^28 sweeps)",
-                                 "l2": "flushed (512 MB write) before every timed call"},
+                                 "l2": L2_NOTE},
                       "roofline": {"bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"],
                                    "peak_source": f"{kind} (HBM copy)"},
                       "cases": cases, "device_status": status}), flush=True)
@@ -762,7 +857,7 @@ def run_codebook_study(args):
     import bit_nf4_quantized_14_b200 as q
     peaks, kind = load_peaks()
     device = torch.device("cuda", 0)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
     x = torch.from_numpy(synth.normal_f32(STUDY_SHAPE, 1.0, 0, 17).reshape(-1)).to(device)
     n = x.numel()
     nf4, _ = q.codebook()
@@ -815,7 +910,7 @@ def run_codebook_study(args):
                       "config": {"workload": "8192 x 8192 N(0, 1) fp32 matrix (2^26 elements), blocks of 64, fp32 "
                                              "constants; codebooks int4 {-7..7}/7, grid {-8..7}/8, NF4, Lloyd "
                                              f"({STUDY_LLOYD_STEPS} device steps from NF4)",
-                                 "l2": "flushed (512 MB write) before every timed codec call; the Lloyd loop runs "
+                                 "l2": L2_NOTE + " (codec calls); the Lloyd loop runs "
                                        "back to back (input 256 MB > L2)"},
                       "roofline": {"bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"],
                                    "peak_source": f"{kind} (HBM copy)"},
@@ -1154,7 +1249,7 @@ def main(argv=None):
                     default="torch",
                     help="with --workload llama65b_train: the adapters' optimizer")
     ap.add_argument("--workload", choices=["llama7b_step", "decode", "codec_sweep", "llama65b_linears",
-                                           "llama65b_train", "codebook_study", "paged_adamw"],
+                                           "llama65b_train", "codebook_study", "paged_adamw", "flush_check"],
                     default="llama7b_step",
                     help="llama7b_step (the headline line), or the decode / codec-sweep / 65B-step measurement lines")
     ap.add_argument("--ncu-summary", metavar="CSV", default=None,
@@ -1186,6 +1281,8 @@ def main(argv=None):
         return run_codebook_study(args)
     if args.workload == "paged_adamw":
         return run_paged_adamw(args)
+    if args.workload == "flush_check":
+        return run_flush_check(args)
     return run_gpu(args)
 
 

@@ -121,6 +121,16 @@ bool build_buckets(const CodebookArg& cb, int nl, BucketArg* out) {
   for (int j = 1; j < nl; ++j)
     if (std::fabs(cb.levels[j]) < std::fabs(cb.levels[z])) z = j;
   out->zero_codes = 0x11111111u * static_cast<uint32_t>(z);
+  // lo(b) as a popcount: lo never drops and rises by at most one from one bucket to the next (two
+  // thresholds inside one bucket's span would share a widened bucket, rejected above)
+  int prev = 0;
+  for (int b = 0; b < 32; ++b) {
+    const int lo = static_cast<int>((out->lo_nibbles[b / 8] >> (4 * (b % 8))) & 0xFu);
+    const int step = lo - prev;
+    if (step < 0 || step > 1) ok = false;
+    else if (step == 1) out->step_mask |= 1u << b;
+    prev = lo;
+  }
   return ok;
 }
 
@@ -495,14 +505,14 @@ GemvWs gemv_ws(int64_t T, int64_t N, int64_t K, int r) {
 }
 
 // ---- decode path (T <= kDcMaxTokens): one cooperative launch of nf4_decode_kernel ---------------
-// Workspace of the decode path (offsets in bytes): one tag per 8-row unit of A, and the per-CTA results
-// awaiting the adapter term when they do not fit in shared memory.
+// Workspace of the decode path (offsets in bytes): one tag per 16-row tile of A, and the per-CTA results
+// awaiting the adapter term when they do not fit in shared memory ([tile][16][T] fp32).
 struct DecWs { size_t tags, base, total; };
 DecWs dec_ws(int64_t T, int64_t N, int r) {
   DecWs w;
   w.tags = 0;
-  w.base = align256(static_cast<size_t>(r / 8) * 8);
-  w.total = w.base + align256(static_cast<size_t>(T) * N * 4);
+  w.base = align256(static_cast<size_t>(cdiv(r, 16)) * 8);
+  w.total = w.base + align256(static_cast<size_t>(cdiv(N, 16)) * 16 * T * 4);
   return w;
 }
 // A value no earlier call in this process used and that uninitialised memory is unlikely to hold: the
@@ -644,36 +654,24 @@ int launch_decode(const void* X, int64_t T, const qlora_nf4_tensor* W, const voi
   if (int e = check_device(&sms)) return e;
   const int64_t N = W->rows, K = W->cols;
   const DecWs L = dec_ws(T, N, r);
-  const int64_t units = N / 8, aunits = r / 8;
-  const int G = static_cast<int>(std::max<int64_t>(
-      1, std::min<int64_t>(units + kDcALoad * aunits, std::min(sms, kGvMaxCtas))));
-  // codes as (32 bytes of a block, row, block); A as (64 elements of a block, row, block); one box height per
-  // pass size
-  const uint64_t nkb = static_cast<uint64_t>(K / 64);
-  DcMaps maps;
-  bool ok = make_tmap_t(&maps.b, B, TmType::kBf16, r, N, r, std::min(r, 64), 8, false);
-  for (int h = 1; ok && h <= kDcUnits; ++h)
-    ok = make_tmap_3d(&maps.c[h - 1], W->codes, TmType::kU8, {32, static_cast<uint64_t>(N), nkb},
-                      {static_cast<uint64_t>(K / 2), 32}, {32, static_cast<uint32_t>(8 * h), kDcStageBlocks}, false);
-  for (int h = 1; ok && h <= kDcAUnits; ++h)
-    ok = make_tmap_3d(&maps.a[h - 1], A, TmType::kBf16, {64, static_cast<uint64_t>(r), nkb},
-                      {static_cast<uint64_t>(K) * 2, 128}, {64, static_cast<uint32_t>(8 * h), kDcStageBlocks}, true);
-  if (!ok) return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
+  const int64_t tiles = cdiv(N, 16), atiles = cdiv(r, 16);
+  const int64_t load = u_only ? kDcALoad * atiles : tiles + kDcALoad * atiles;
+  const int G = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(load, std::min(sms, kGvMaxCtas))));
   DecParams p{};
   p.T = static_cast<int>(T); p.N = static_cast<int>(N); p.K = static_cast<int>(K); p.r = r;
   p.RP = static_cast<int>(cdiv(r, 64) * 64);
   p.nkb = static_cast<int>(K / 64);
-  p.units = static_cast<int>(units);
-  p.aunits = static_cast<int>(aunits);
+  p.tiles = static_cast<int>(tiles);
+  p.atiles = static_cast<int>(atiles);
   p.u_only = u_only ? 1 : 0;
-  // the most NF4 units one CTA can get (see dc_share): ceil(L / G) load positions
-  const int64_t per_cta = cdiv(units + kDcALoad * aunits, G);
-  p.base_in_smem = per_cta * T * 8 * 4 <= kDcBaseBytes ? 1 : 0;
   p.s = s;
   p.X = static_cast<const __nv_bfloat16*>(X);
+  p.codes = W->codes;
   p.e4m3 = W->absmax_e4m3;
   p.s2 = W->scale2;
   p.mu = W->offset;
+  p.A = static_cast<const __nv_bfloat16*>(A);
+  p.B = static_cast<const __nv_bfloat16*>(B);
   p.Y = static_cast<__nv_bfloat16*>(Y);
   p.U = static_cast<__nv_bfloat16*>(U);
   p.tags = reinterpret_cast<uint64_t*>(dws + L.tags);
@@ -692,7 +690,7 @@ int launch_decode(const void* X, int64_t T, const qlora_nf4_tensor* W, const voi
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, maps, p, codebook()) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, kern, p, codebook()) != cudaSuccess)
     return cuda_fail(cudaGetLastError(), "cooperative launch", __LINE__);
   return launched();
 }
@@ -772,6 +770,32 @@ int noalloc_scratch(void** out) {
   return QLORA_OK;
 }
 
+// Pass 1 on stream st: persistent, Q1<InT>::kCtasPerSm CTAs per SM (fewer when there are fewer whole slabs).
+// With ssum and ticket null it writes the fp32 constants as they are (the single-quantization format).
+template <typename InT>
+int launch_pass1_t(const InT* w, int64_t n, uint8_t* codes, float* c1, double* ssum, unsigned* ticket,
+                   const CodebookArg& cb, const BucketArg& bk, int sms, cudaStream_t st) {
+  if (cudaFuncSetAttribute(nf4_quantize_pass1<InT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           Q1<InT>::kSmemBytes) != cudaSuccess)
+    return cuda_fail(cudaGetLastError(), "cudaFuncSetAttribute", __LINE__);
+  const int64_t nfull = n / kSlabElems;
+  const unsigned grid =
+      static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(nfull, int64_t(sms) * Q1<InT>::kCtasPerSm)));
+  nf4_quantize_pass1<InT><<<grid, kQ1Threads, Q1<InT>::kSmemBytes, st>>>(w, n, codes, c1, ssum, cdiv(n, kSlabElems),
+                                                                          cb, bk, ticket);
+  return launched();
+}
+int launch_pass1(const void* w, int w_dtype, int64_t n, uint8_t* codes, float* c1, double* ssum, unsigned* ticket,
+                 const CodebookArg& cb, const BucketArg& bk, int sms, cudaStream_t st) {
+  if (w_dtype == QLORA_F32)
+    return launch_pass1_t(static_cast<const float*>(w), n, codes, c1, ssum, ticket, cb, bk, sms, st);
+  const unsigned grid = static_cast<unsigned>(
+      std::max<int64_t>(1, std::min<int64_t>(cdiv(cdiv(n, kSlabElems), kQuantThreads / 32), int64_t(sms) * kQuantMinBlocks)));
+  nf4_quantize_pass1_direct<__nv_bfloat16><<<grid, kQuantThreads, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(w), n, codes, c1, ssum, cdiv(n, kSlabElems), cb, bk, ticket);
+  return launched();
+}
+
 // Passes 1, 1b and 2 of the quantizer on stream st, workspace laid out by quant_ws(n).
 int run_quantize(const void* w, int w_dtype, int64_t n, const qlora_nf4_tensor* out, void* ws, cudaStream_t st) {
   int sms = 0;
@@ -785,16 +809,7 @@ int run_quantize(const void* w, int w_dtype, int64_t n, const qlora_nf4_tensor* 
   double* partial = reinterpret_cast<double*>(base + L.partial);
   unsigned* ticket = reinterpret_cast<unsigned*>(base + L.ticket);
   const int64_t nb = cdiv(n, kBlock), ng = cdiv(nb, kGroup);
-  const unsigned g1 = static_cast<unsigned>(
-      std::min<int64_t>(cdiv(L.nslabs, kQuantThreads / 32), int64_t(sms) * kQuantMinBlocks));
-  if (w_dtype == QLORA_F32)
-    nf4_quantize_pass1<float><<<g1, kQuantThreads, 0, st>>>(static_cast<const float*>(w), n, out->codes, c1, ssum,
-                                                             L.nslabs, codebook(), bk.arg, ticket);
-  else
-    nf4_quantize_pass1<__nv_bfloat16><<<g1, kQuantThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(w), n,
-                                                                     out->codes, c1, ssum, L.nslabs, codebook(),
-                                                                     bk.arg, ticket);
-  if (int e = launched()) return e;
+  if (int e = launch_pass1(w, w_dtype, n, out->codes, c1, ssum, ticket, codebook(), bk.arg, sms, st)) return e;
   if (launch_pdl(nf4_mean, L.mean_ctas, kTreeThreads, st, ssum, L.nslabs, nb, partial, ticket, out->offset) !=
       cudaSuccess)
     return cuda_fail(cudaGetLastError(), "CUDA call or tensor-map encode", __LINE__);
@@ -825,16 +840,7 @@ int launch_dequant(bool bf16, bool single, const uint8_t* codes, const uint8_t* 
 // Pass 1 alone, with fp32 block constants kept as they are (no slab sums, no mean pass).
 int launch_pass1_single(const void* w, int w_dtype, int64_t n, uint8_t* codes, float* absmax,
                         const CodebookArg& cb, const BucketArg& bk, int sms, cudaStream_t st) {
-  const int64_t ns = cdiv(n, kSlabElems);
-  const unsigned g1 =
-      static_cast<unsigned>(std::min<int64_t>(cdiv(ns, kQuantThreads / 32), int64_t(sms) * kQuantMinBlocks));
-  if (w_dtype == QLORA_F32)
-    nf4_quantize_pass1<float><<<g1, kQuantThreads, 0, st>>>(static_cast<const float*>(w), n, codes, absmax,
-                                                             nullptr, ns, cb, bk, nullptr);
-  else
-    nf4_quantize_pass1<__nv_bfloat16><<<g1, kQuantThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(w), n, codes,
-                                                                     absmax, nullptr, ns, cb, bk, nullptr);
-  return launched();
+  return launch_pass1(w, w_dtype, n, codes, absmax, nullptr, nullptr, cb, bk, sms, st);
 }
 
 static_assert(kStatOut == QLORA_CODEBOOK_STATS_LEN, "codebook statistics layout");

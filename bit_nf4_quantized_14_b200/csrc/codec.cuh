@@ -41,6 +41,7 @@ struct CodebookArg {       // passed by value: lives in the kernel-parameter con
 struct BucketArg {         // bucket b -> lo(b), 4 bits each; the code of an all-zero block in every nibble
   uint32_t lo_nibbles[4];
   uint32_t zero_codes;
+  uint32_t step_mask;      // bit b = lo(b) - lo(b - 1) (bit 0 = lo(0)): lo(b) = popc(bits 0..b)
 };
 
 constexpr int kBlock = 64;          // first-level block (weights per absmax constant)
@@ -49,8 +50,6 @@ constexpr int kGroupElems = kBlock * kGroup;
 constexpr int kSlabBlocks = 64;     // pass 1: one warp owns a slab of 64 blocks
 constexpr int kSlabElems = kSlabBlocks * kBlock;
 constexpr int kStepElems = 512;     // one warp step: 8 blocks, 16 elements per lane
-constexpr int kQuantThreads = 256;
-constexpr int kQuantMinBlocks = 3;
 constexpr float kBucketScale = 15.0f;
 constexpr float kBucketBias = 12582928.0f;   // 1.5 * 2^23 + 16
 constexpr double kBucketWiden = 0x1p-18;     // table margin in units of t
@@ -112,26 +111,27 @@ template <> struct Raw16<__nv_bfloat16> {
   }
 };
 
-// Code of one element. lotab: lane b holds lo(b) (as raw bits); ttab: lane j holds T_j, lanes >= 15 +inf.
+// Code of one element. tbtab: lane b holds T_lo(b), the one threshold that can lie in bucket b (+inf when
+// lo(b) = 15 or the codebook has fewer thresholds); lo(b) = popc(bits 0..b of the step mask). The bucket's
+// shuffle and the popcount do not depend on each other.
 template <bool kScaled>
-__device__ __forceinline__ uint32_t nf4_code(float x, float a, float sc, float r15, float lotab, float ttab) {
+__device__ __forceinline__ uint32_t nf4_code(float x, float a, float sc, float r15, float tbtab, uint32_t step_mask) {
   const float xs = kScaled ? x * sc : x;
-  const float z = __fmaf_rn(xs, r15, kBucketBias);
-  const uint32_t lo =
-      __float_as_uint(__shfl_sync(0xffffffffu, lotab, static_cast<int>(__float_as_uint(z))));
-  const float tl = __shfl_sync(0xffffffffu, ttab, static_cast<int>(lo));
+  const uint32_t zb = __float_as_uint(__fmaf_rn(xs, r15, kBucketBias));   // bucket in the low 5 bits
+  const float tl = __shfl_sync(0xffffffffu, tbtab, static_cast<int>(zb));
+  const uint32_t lo = __popc(step_mask << (~zb & 31u));
   return lo + ((x > __fmul_rd(tl, a)) ? 1u : 0u);
 }
 // Codes of 16 elements as 8 bytes, byte i = (code[2i] << 4) | code[2i+1] (even element high nibble).
 template <bool kScaled>
-__device__ __forceinline__ void nf4_codes16(const float (&x)[16], float a, float sc, float r15, float lotab,
-                                            float ttab, uint32_t& w0, uint32_t& w1) {
+__device__ __forceinline__ void nf4_codes16(const float (&x)[16], float a, float sc, float r15, float tbtab,
+                                            uint32_t step_mask, uint32_t& w0, uint32_t& w1) {
   w0 = 0;
   w1 = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint32_t hi = nf4_code<kScaled>(x[2 * i], a, sc, r15, lotab, ttab);
-    const uint32_t lo = nf4_code<kScaled>(x[2 * i + 1], a, sc, r15, lotab, ttab);
+    const uint32_t hi = nf4_code<kScaled>(x[2 * i], a, sc, r15, tbtab, step_mask);
+    const uint32_t lo = nf4_code<kScaled>(x[2 * i + 1], a, sc, r15, tbtab, step_mask);
     const uint32_t b = (hi << 4) | lo;
     if (i < 4) w0 |= b << (8 * i);
     else w1 |= b << (8 * (i - 4));
@@ -140,7 +140,7 @@ __device__ __forceinline__ void nf4_codes16(const float (&x)[16], float a, float
 
 // One step of a warp: lanes 4k..4k+3 hold block k's 64 elements (16 each). Returns the team's absmax
 // (NaN if the block holds a NaN); flags a non-finite block in `bad`.
-__device__ __forceinline__ float block_codes(const float (&x)[16], float lotab, float ttab, uint32_t zero_codes,
+__device__ __forceinline__ float block_codes(const float (&x)[16], float tbtab, uint32_t step_mask, uint32_t zero_codes,
                                              uint32_t& bad, uint32_t& w0, uint32_t& w1) {
   float m = fmax_nan(fmax_nan(fmax_nan(fabsf(x[0]), fabsf(x[1])), fmax_nan(fabsf(x[2]), fabsf(x[3]))),
                      fmax_nan(fmax_nan(fabsf(x[4]), fabsf(x[5])), fmax_nan(fabsf(x[6]), fabsf(x[7]))));
@@ -153,8 +153,8 @@ __device__ __forceinline__ float block_codes(const float (&x)[16], float lotab, 
   const bool tiny = a < 0x1p-120f;
   const float sc = tiny ? 0x1p64f : 1.0f;
   const float r15 = kBucketScale * rcp_approx(a * sc);
-  if (__any_sync(0xffffffffu, tiny)) nf4_codes16<true>(x, a, sc, r15, lotab, ttab, w0, w1);
-  else nf4_codes16<false>(x, a, sc, r15, lotab, ttab, w0, w1);
+  if (__any_sync(0xffffffffu, tiny)) nf4_codes16<true>(x, a, sc, r15, tbtab, step_mask, w0, w1);
+  else nf4_codes16<false>(x, a, sc, r15, tbtab, step_mask, w0, w1);
   if (!(a > 0.0f)) {                                // all-zero block (or NaN): the zero code
     w0 = zero_codes;
     w1 = zero_codes;
@@ -162,19 +162,175 @@ __device__ __forceinline__ float block_codes(const float (&x)[16], float lotab, 
   return a;
 }
 
-// Pass 1. Each warp owns slabs gw, gw + nw, ... and walks them as a flat sequence of 8-block steps,
-// loading step i+1 while step i computes. Per slab it writes the 64 block constants (fp32) and their
-// fp64 balanced-tree sum. A ragged last slab is done by one warp at the end, with bounds on every element.
-// Without double quantization (ssum and ticket null) c1 is the stored constant array and pass 1 is all.
+// Pass 1 for fp32 input. Persistent CTAs, two per SM; CTA c owns a contiguous range of whole slabs. One
+// producer lane brings each slab into a ring of shared-memory slots with one bulk copy (a ring of 96 KB per CTA keeps
+// ~190 KB per SM in flight, what HBM needs to stay busy); consumer warp w takes step w (blocks 8w..8w+7)
+// of every slab, writes its codes straight to global memory and its 8 constants to the slot's constant
+// buffer, and the last of the eight warps to finish a slab (a shared-memory counter) writes the slab's
+// 64 constants and their fp64 balanced-tree sum. A ragged last slab is done by one warp of the last CTA
+// with direct loads and bounds on every element. Without double quantization (ssum and ticket null) c1
+// is the stored constant array and pass 1 is all.
+template <typename InT> struct Q1 {
+  static constexpr int kSlabBytes = kSlabElems * static_cast<int>(sizeof(InT));
+  static constexpr int kCtasPerSm = 2;
+  static constexpr int kSlots = (96 * 1024) / kSlabBytes;
+  static constexpr int kOffCb = kSlots * kSlabBytes;                      // [slot][64] fp32 constants
+  static constexpr int kOffCnt = kOffCb + kSlots * kSlabBlocks * 4;       // [slot] finished-warp counters
+  static constexpr int kOffBar = kOffCnt + kSlots * 4 + 8 - (kSlots * 4) % 8;
+  static constexpr int kOffRag = kOffBar + 2 * kSlots * 8;                // full[slot], empty[slot]
+  static constexpr int kSmemBytes = kOffRag + kSlabBlocks * 4;            // the ragged slab's constants
+};
+constexpr int kQ1Consumers = 8;                       // = steps per slab
+constexpr int kQ1Threads = 32 * (kQ1Consumers + 1);
+static_assert(kQ1Consumers * kStepElems == kSlabElems, "one step per consumer warp");
+
+// One lane's 16 elements of a slab slot: this lane's 64 contiguous bytes are read in
+// 16-byte chunks starting at a lane-dependent chunk, so every 128-byte wavefront serves 8 distinct lanes
+// (no bank conflicts); the chunks land rotated and the packed codes are rotated back.
+template <typename InT> struct SlotRead;
+template <> struct SlotRead<float> {
+  static __device__ __forceinline__ int rot(int lane) { return (lane >> 1) & 3; }
+  static __device__ __forceinline__ void load(const uint8_t* p, int r, float (&x)[16]) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 v = *reinterpret_cast<const uint4*>(p + 16 * ((c + r) & 3));
+      x[4 * c] = __uint_as_float(v.x); x[4 * c + 1] = __uint_as_float(v.y);
+      x[4 * c + 2] = __uint_as_float(v.z); x[4 * c + 3] = __uint_as_float(v.w);
+    }
+  }
+  static __device__ __forceinline__ uint2 unrotate(uint32_t w0, uint32_t w1, int r) {   // 16-bit pieces
+    const uint64_t v = (static_cast<uint64_t>(w1) << 32) | w0;
+    const uint64_t o = r ? ((v << (16 * r)) | (v >> (64 - 16 * r))) : v;
+    return make_uint2(static_cast<uint32_t>(o), static_cast<uint32_t>(o >> 32));
+  }
+};
 template <typename InT>
-__global__ void __launch_bounds__(kQuantThreads, kQuantMinBlocks) nf4_quantize_pass1(
+__global__ void __launch_bounds__(kQ1Threads, Q1<InT>::kCtasPerSm) nf4_quantize_pass1(
+    const InT* __restrict__ w, int64_t n, uint8_t* __restrict__ codes, float* __restrict__ c1,
+    double* __restrict__ ssum, int64_t nslabs, CodebookArg cb, BucketArg bk, unsigned* __restrict__ ticket) {
+  using L = Q1<InT>;
+  extern __shared__ __align__(1024) uint8_t q1_smem[];
+  float* cbuf = reinterpret_cast<float*>(q1_smem + L::kOffCb);
+  unsigned* cnt = reinterpret_cast<unsigned*>(q1_smem + L::kOffCnt);
+  uint64_t* full = reinterpret_cast<uint64_t*>(q1_smem + L::kOffBar);
+  uint64_t* empty = full + L::kSlots;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (ticket && blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0u;    // arrival counter of the mean pass
+  const int64_t nb = (n + kBlock - 1) / kBlock;
+  const int64_t nfull = n / kSlabElems;
+  const int64_t s0 = nfull * blockIdx.x / gridDim.x, s1 = nfull * (blockIdx.x + 1) / gridDim.x;
+  const int nmine = static_cast<int>(s1 - s0);
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < L::kSlots; ++k) {
+      mbar_init(&full[k], 1);
+      mbar_init(&empty[k], kQ1Consumers + 1);     // the eight readers and the slab's finisher
+      cnt[k] = 0u;
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  // constants out, and the slab's 64-leaf fp64 tree (leaf pairs per lane, then a butterfly of subtrees)
+  auto finish_slab = [&](int64_t s, const float* cbs) {
+    const float l0 = cbs[2 * lane], l1 = cbs[2 * lane + 1];
+    const int64_t gb = s * kSlabBlocks + 2 * lane;
+    if (gb + 1 < nb) *reinterpret_cast<float2*>(c1 + gb) = make_float2(l0, l1);
+    else if (gb < nb) c1[gb] = l0;
+    double t = static_cast<double>(l0) + static_cast<double>(l1);
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const double r = __shfl_down_sync(0xffffffffu, t, off);
+      if ((lane & (2 * off - 1)) == 0) t = t + r;    // left subtree + right subtree
+    }
+    if (lane == 0 && ssum) ssum[s] = t;
+  };
+
+  if (warp == kQ1Consumers) {                     // producer
+    if (lane == 0) {
+      for (int i = 0; i < nmine; ++i) {
+        const int k = i % L::kSlots;
+        if (i >= L::kSlots && !mbar_wait(&empty[k], ((i / L::kSlots) - 1) & 1)) break;
+        mbar_arrive_expect_tx(&full[k], L::kSlabBytes);
+        bulk_load(q1_smem + k * L::kSlabBytes, w + (s0 + i) * kSlabElems, L::kSlabBytes, &full[k]);
+      }
+    }
+  } else {
+    const uint32_t lo_lane = (bk.lo_nibbles[lane >> 3] >> (4 * (lane & 7))) & 0xFu;
+    const float tbtab = (lo_lane < 15) ? cb.thresholds[lo_lane] : __int_as_float(0x7F800000);
+    const int rot = SlotRead<InT>::rot(lane);
+    uint32_t bad = 0;
+    for (int i = 0; i < nmine; ++i) {
+      const int k = i % L::kSlots;
+      if (!mbar_wait(&full[k], (i / L::kSlots) & 1)) break;
+      float x[16];
+      SlotRead<InT>::load(q1_smem + k * L::kSlabBytes + (warp * kStepElems + 16 * lane) * sizeof(InT), rot, x);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[k]);
+      uint32_t w0, w1;
+      const float a = block_codes(x, tbtab, bk.step_mask, bk.zero_codes, bad, w0, w1);
+      const int64_t s = s0 + i;
+      *reinterpret_cast<uint2*>(codes + ((s * kSlabElems + warp * kStepElems + 16 * lane) >> 1)) =
+          SlotRead<InT>::unrotate(w0, w1, rot);
+      float* cbs = cbuf + k * kSlabBlocks;
+      if ((lane & 3) == 0) cbs[warp * 8 + (lane >> 2)] = a;
+      __threadfence_block();
+      __syncwarp();
+      unsigned last = 0;
+      if (lane == 0) last = (atomicAdd(&cnt[k], 1u) == kQ1Consumers - 1) ? 1u : 0u;
+      if (__shfl_sync(0xffffffffu, last, 0)) {    // the last warp of this slab: publish it
+        __threadfence_block();
+        finish_slab(s, cbs);
+        __syncwarp();
+        if (lane == 0) {
+          cnt[k] = 0u;
+          mbar_arrive(&empty[k]);
+        }
+      }
+    }
+    if (nfull < nslabs && blockIdx.x == gridDim.x - 1 && warp == 0) {   // the ragged last slab
+      const int64_t s = nfull;
+      float* cbs = reinterpret_cast<float*>(q1_smem + L::kOffRag);
+      for (int it = 0; it < kSlabElems / kStepElems; ++it) {
+        const int64_t e0 = s * kSlabElems + it * kStepElems + 16 * lane;
+        float x[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x[e] = (e0 + e < n) ? Scalar<InT>::load(w + e0 + e) : 0.0f;
+        uint32_t w0, w1;
+        const float a = block_codes(x, tbtab, bk.step_mask, bk.zero_codes, bad, w0, w1);
+        for (int b = 0; b < 8; ++b) {
+          const int64_t idx = e0 + 2 * b;
+          if (idx < n) {
+            uint32_t byte = ((b < 4 ? w0 : w1) >> (8 * (b & 3))) & 0xFFu;
+            if (idx + 1 >= n) byte &= 0xF0u;                     // odd n: the final low nibble is 0
+            codes[idx >> 1] = static_cast<uint8_t>(byte);
+          }
+        }
+        if ((lane & 3) == 0) cbs[it * 8 + (lane >> 2)] = a;
+      }
+      __syncwarp();
+      finish_slab(s, cbs);
+    }
+    if (bad) raise_status(kStatusNonfinite);
+  }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Pass 1 for bf16 input. Each warp owns slabs gw, gw + nw, ... and walks them as a flat sequence of
+// 8-block steps straight from global memory, loading step i + 1 while step i computes (three CTAs of eight
+// warps per SM: half the bytes per element of fp32 input leave the issue rate, not HBM, as the limit, and
+// more warps per SM serve it better than a shared-memory ring). Per slab it writes the 64 block constants
+// and their fp64 balanced-tree sum; a ragged last slab is done by one warp with bounds on every element.
+constexpr int kQuantThreads = 256;
+constexpr int kQuantMinBlocks = 3;
+template <typename InT>
+__global__ void __launch_bounds__(kQuantThreads, kQuantMinBlocks) nf4_quantize_pass1_direct(
     const InT* __restrict__ w, int64_t n, uint8_t* __restrict__ codes, float* __restrict__ c1,
     double* __restrict__ ssum, int64_t nslabs, CodebookArg cb, BucketArg bk, unsigned* __restrict__ ticket) {
   __shared__ float c1buf[kQuantThreads / 32][kSlabBlocks];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (ticket && blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0u;    // arrival counter of the mean pass
-  const float lotab = __uint_as_float((bk.lo_nibbles[lane >> 3] >> (4 * (lane & 7))) & 0xFu);
-  const float ttab = (lane < 15) ? cb.thresholds[lane] : __int_as_float(0x7F800000);
+  const uint32_t lo_lane = (bk.lo_nibbles[lane >> 3] >> (4 * (lane & 7))) & 0xFu;
+  const float tbtab = (lo_lane < 15) ? cb.thresholds[lo_lane] : __int_as_float(0x7F800000);
   const int64_t nb = (n + kBlock - 1) / kBlock;
   const int64_t nfull = n / kSlabElems;
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * (kQuantThreads / 32) + warp;
@@ -212,7 +368,7 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinBlocks) nf4_quantize_p
     cur.widen(x);
     const int64_t e0 = s * kSlabElems + it * kStepElems + 16 * lane;
     uint32_t w0, w1;
-    const float a = block_codes(x, lotab, ttab, bk.zero_codes, bad, w0, w1);
+    const float a = block_codes(x, tbtab, bk.step_mask, bk.zero_codes, bad, w0, w1);
     *reinterpret_cast<uint2*>(codes + (e0 >> 1)) = make_uint2(w0, w1);
     if ((lane & 3) == 0) cb_w[it * 8 + (lane >> 2)] = a;
     if (it == 7) finish_slab(s);
@@ -225,7 +381,7 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinBlocks) nf4_quantize_p
 #pragma unroll
       for (int e = 0; e < 16; ++e) x[e] = (e0 + e < n) ? Scalar<InT>::load(w + e0 + e) : 0.0f;
       uint32_t w0, w1;
-      const float a = block_codes(x, lotab, ttab, bk.zero_codes, bad, w0, w1);
+      const float a = block_codes(x, tbtab, bk.step_mask, bk.zero_codes, bad, w0, w1);
       for (int b = 0; b < 8; ++b) {
         const int64_t idx = e0 + 2 * b;
         if (idx < n) {

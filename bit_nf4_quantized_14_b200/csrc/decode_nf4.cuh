@@ -1,33 +1,36 @@
 // Decode-sized QLoRA forward (T <= 16 tokens), one launch:
 //     Y = X W_hat^T + sU B^T,   sU = s X A^T   (s = alpha / r),
-// with W stored as NF4 codes plus double-quantized block constants. The weight is "dequantized to
-// bfloat16 on the fly, block by block, and multiplied in 16-bit precision" (PEFT page,
-// zerotofrontier.app/sft/peft, "Paged optimizers, and QLoRA end to end"), inside the matrix multiply
-// (same page, "The real way"); the adapter term is the explainer's X L1 L2 (QLoRA explainer,
-// prism.theerrors.in, "Putting it together").
+// with W stored as NF4 codes plus double-quantized block constants. The weight is expanded to bf16 block
+// by block while the contraction consumes it and multiplied in 16-bit arithmetic (PEFT page,
+// zerotofrontier.app/sft/peft, "Paged optimizers, and QLoRA end to end"; the fused form: same page, "The
+// real way"); the adapter term is the explainer's X L1 L2 (QLoRA explainer, prism.theerrors.in, "Putting
+// it together").
 //
 // With a handful of tokens every weight is used T times, so the layer is bound by streaming 0.52 B per
 // weight from HBM. The design keeps the per-weight work to two instructions (a byte permute and a
-// shared-memory load per two weights) and moves everything else off that path:
-//   * persistent grid, one CTA per SM (cooperative launch: every CTA resident). The rows of W (in units
-//     of 8) and the rows of A (the adapter projection, also in units of 8, each weighted 4x for its 4x
-//     bytes per element) are split into contiguous ranges, one per CTA; each CTA contracts its units over
-//     the whole K, so no partial sum crosses CTAs;
-//   * a TMA ring of stages, each 16 blocks (1024 contraction elements) of up to 8 NF4 units or 2 A units,
-//     one three-dimensional box per stage (block, row, bytes of the block): codes land as
-//     [block][row][32 B], which the fragment loads read without bank conflicts, and A rows as
-//     [block][row][128 B] with the 128-byte swizzle; consumer warp w takes block w of every stage;
-//   * mma.sync m16n8k16: the A operand is X (16 token rows, padded), the B operand is 8 rows of one
-//     64-element block. For NF4 rows it is built from code bytes: prmt forms (byte << 8 | lane * 4) and one
-//     shared-memory load fetches the bf16 pair (level[hi], level[lo]) from a 256-entry table replicated
-//     per lane (entries 256 B apart, so the address needs no further arithmetic and never conflicts);
-//   * the block constant c1_hat = fma(decode(e4m3), s2, mu) multiplies the fp32 result of each block's
-//     four MMAs; a scale warp computes the stage's constants one stage ahead;
+// shared-memory load per two weights) and keeps the HBM stream out of shared memory:
+//   * persistent grid, one CTA per SM (cooperative launch: every CTA resident). The rows of W and of A
+//     (the adapter projection), in tiles of 16 rows, are split into contiguous ranges, one per CTA (an A
+//     tile weighs 4 NF4 tiles: bf16 against 4-bit); each CTA contracts its tiles over the whole K, so no
+//     partial sum crosses CTAs;
+//   * passes of up to 4 tiles (2 for more than 8 tokens), each a sequence of stages of 16 blocks (1024
+//     contraction elements); consumer warp w takes block w of every stage. Each warp streams its own bytes
+//     (block w of the pass's rows, 32-byte sectors used whole) into a private ring of 4 shared-memory slots
+//     with cp.async, three stages ahead, so ~96 KB per SM are in flight without holding registers, and no
+//     warp waits for another to refill a slot;
+//   * mma.sync m16n8k16 with the weight as the 16-row A operand and X as the 8-token B operand. The A
+//     fragments come from code bytes: prmt forms (byte << 8 | lane * 4) and one shared-memory load fetches
+//     the bf16 pair (level[hi], level[lo]) from a 256-entry table replicated per lane (entries 256 B
+//     apart: no further arithmetic, no bank conflicts). Inside each 64-element block the MMA's k index is
+//     permuted (the same permutation on both operands) so lane j's 16 elements are 16 j .. 16 j + 15;
+//   * the block constant c1_hat = fma(decode(e4m3), s2, mu) multiplies the fp32 result of each block's four
+//     MMAs; a helper warp decodes each stage's constants into a ring of shared-memory buffers ahead of the
+//     consumers, from raw bytes it loads three stages ahead;
 //   * at the end of each pass the 16 warps' partial sums meet in shared memory and are added in warp
-//     order (deterministic). A units come first: their sums, times s and rounded to bf16, are sU, which
-//     the CTA publishes with a per-call tag; a gather warp in every CTA waits for all of sU and copies it
-//     into shared memory, and the adapter term sU B^T is one more contraction per unit at the end, against
-//     B rows brought in by TMA.
+//     order (deterministic). A tiles come first: their sums, times s and rounded to bf16, are sU, which the
+//     CTA publishes with a per-call tag; a gather warp in every CTA waits for all of sU and copies it into
+//     shared memory, and the adapter term sU B^T is one more contraction per tile at the end, with B rows
+//     loaded straight into the MMA's A operand.
 // The one difference from the fused GEMM's W_hat = bf16(level * c1_hat) is where the bf16 rounding falls
 // (on the level instead of the product): both round each weight once, to a relative 2^-9.
 // sU's summation order depends only on K (not on the grid), and the backward recomputes it with this
@@ -36,70 +39,58 @@
 // unwinds without further waits. Named barriers among the consumer warps are reached on every path.
 #pragma once
 
-#include <cuda.h>
-
 #include "codec.cuh"
 #include "common.cuh"
 
 namespace qnf4 {
 
 constexpr int kDcWarps = 16;                          // consumer warps: warp w takes block w of a stage
-constexpr int kDcThreads = 32 * (kDcWarps + 2);       // + scale/TMA warp + gather warp
-constexpr int kDcUnits = 8;                           // NF4 units per pass (8 rows each)
-constexpr int kDcAUnits = 2;                          // A units per pass
-constexpr int kDcALoad = 4;                           // an A unit weighs as much as 4 NF4 units
-constexpr int kDcStages = 4;                          // ring slots
-constexpr int kDcStageBlocks = 16;
-constexpr int kDcSlotBytes = 32 * 1024;               // NF4: [col box 0..3][unit 0..7]; A: [unit][block]
-constexpr int kDcLutBytes = 256 * 256;                // entry e at e * 256: lane copies in bytes 0..127
-constexpr int kDcCbufBytes = kDcStageBlocks * 4 * kDcUnits * 2 * 4;   // [block][j][unit][2] fp32
+constexpr int kDcThreads = 32 * (kDcWarps + 2);       // + constants warp + gather warp
+constexpr int kDcMaxTiles = 4;                        // NF4 tiles per pass (2 when T > 8)
+constexpr int kDcALoad = 4;                           // an A tile weighs as much as 4 NF4 tiles
+constexpr int kDcStageBlocks = kDcWarps;
+constexpr int kDcRing = 4;                            // code slots per consumer warp
+constexpr int kDcWarpSlot = 2048;                     // one stage of one warp: 64 rows x 32 B, or 16 A rows x 128 B
+constexpr int kDcCRing = 4;                           // constant buffers (stages) in flight
 constexpr int kDcMaxTokens = 16;
 constexpr int kDcMaxRank = 256;
+constexpr int kDcLutBytes = 256 * 256;                // entry e at e * 256: lane copies in bytes 0..127
 constexpr int kDcOffRing = kDcLutBytes;
-constexpr int kDcOffCbuf = kDcOffRing + kDcStages * kDcSlotBytes;
-constexpr int kDcOffSU = kDcOffCbuf + 2 * kDcCbufBytes;
+constexpr int kDcCbufBytes = kDcStageBlocks * kDcMaxTiles * 8 * 8;   // [block][tile][g] (row g, row g + 8)
+constexpr int kDcOffCbuf = kDcOffRing + kDcWarps * kDcRing * kDcWarpSlot;
+constexpr int kDcOffSU = kDcOffCbuf + kDcCRing * kDcCbufBytes;
 constexpr int kDcSUBytes = kDcMaxTokens * kDcMaxRank * 2;
-constexpr int kDcOffBase = kDcOffSU + kDcSUBytes;
-constexpr int kDcSmemBytes = 227 * 1024;
-constexpr int kDcOffBar = kDcSmemBytes - 256;
-constexpr int kDcBaseBytes = kDcOffBar - kDcOffBase;  // per-CTA fp32 results awaiting the adapter term
-static_assert(kDcBaseBytes >= 16 * 1024, "shared-memory budget");
-static_assert(kDcAUnits * kDcStageBlocks * 1024 <= kDcSlotBytes, "an A stage fits a slot");
+constexpr int kDcOffBar = kDcOffSU + kDcSUBytes;
+constexpr int kDcSmemBytes = kDcOffBar + 128;
+static_assert(kDcSmemBytes <= 227 * 1024, "shared-memory budget");
 
 struct DecParams {
   int T, N, K, r, RP;        // RP: r rounded up to 64
   int nkb;                   // K / 64
-  int units;                 // N / 8: NF4 units
-  int aunits;                // r / 8: A units
+  int tiles;                 // ceil(N / 16): NF4 tiles
+  int atiles;                // ceil(r / 16): A tiles
   int u_only;                // 1: compute sU only (the backward's recompute)
-  int base_in_smem;          // per-CTA fp32 results fit in shared memory
   float s;
   const __nv_bfloat16* X;    // T x K
+  const uint8_t* codes;      // N x K / 2
   const uint8_t* e4m3;       // N * K / 64
   const float* s2;
   const float* mu;
+  const __nv_bfloat16* A;    // r x K
+  const __nv_bfloat16* B;    // N x r
   __nv_bfloat16* Y;          // T x N
   __nv_bfloat16* U;          // T x r: sU in bf16
-  uint64_t* tags;            // one per A unit
-  float* base_ws;            // [unit][T][8] fp32 when the shared copy does not fit
+  uint64_t* tags;            // one per A tile
+  float* base_ws;            // [tile][16][T] fp32: NF4 results awaiting the adapter term
   uint64_t seq;              // this call's tag value
 };
 
-// Tensor maps of one call: codes as (32 bytes of a block, row, block) with a box height for every
-// pass size of 1..8 units; A as (64 elements of a block, row, block) for passes of 1 or 2 units
-// (128-byte swizzle); B as (r elements, row) for the adapter stages.
-struct DcMaps {
-  CUtensorMap c[kDcUnits];
-  CUtensorMap a[kDcAUnits];
-  CUtensorMap b;
-};
-
-__device__ __forceinline__ void dc_mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
-                                       uint32_t b1) {
+__device__ __forceinline__ void dc_mma(float& d0, float& d1, float& d2, float& d3, uint32_t a0, uint32_t a1,
+                                       uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "+f"(d0), "+f"(d1), "+f"(d2), "+f"(d3)
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 __device__ __forceinline__ uint32_t dc_prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -113,11 +104,24 @@ __device__ __forceinline__ uint32_t dc_prmt(uint32_t a, uint32_t b, uint32_t sel
 __device__ __forceinline__ uint32_t dc_ld32(const uint8_t* sm, uint32_t off) {
   return *reinterpret_cast<const uint32_t*>(sm + off);
 }
-__device__ __forceinline__ uint2 dc_ld64(const uint8_t* sm, uint32_t off) {
-  return *reinterpret_cast<const uint2*>(sm + off);
+__device__ __forceinline__ float2 dc_ldf2(const uint8_t* sm, uint32_t off) {
+  return *reinterpret_cast<const float2*>(sm + off);
 }
 __device__ __forceinline__ uint4 dc_ld128(const uint8_t* sm, uint32_t off) {
   return *reinterpret_cast<const uint4*>(sm + off);
+}
+__device__ __forceinline__ uint2 dc_ld64(const uint8_t* sm, uint32_t off) {
+  return *reinterpret_cast<const uint2*>(sm + off);
+}
+// 16 bytes global -> shared through L2 only (cp.async.cg); src_bytes 0 writes 16 zero bytes and reads
+// nothing. Completion is tracked per thread in commit groups.
+__device__ __forceinline__ void dc_cp16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void dc_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int kPending>
+__device__ __forceinline__ void dc_cp_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
 }
 __device__ __forceinline__ void dc_bar_consumers() {   // the 16 consumer warps only
   asm volatile("bar.sync 1, %0;" ::"n"(32 * kDcWarps) : "memory");
@@ -131,62 +135,35 @@ __device__ __forceinline__ uint32_t dc_pair(const uint8_t* sm, uint32_t w, uint3
 __device__ __forceinline__ float* dc_red(uint8_t* sm, int idx) {
   return reinterpret_cast<float*>(sm + ((idx >> 5) << 8) + 128 + ((idx & 31) << 2));
 }
-// X operand fragments of one 64-element block for token rows g and g + 8 (clamped to T - 1; rows past
-// T repeat the last token and their results are discarded): elements 16 j .. 16 j + 15 of the block.
-template <int TT>
-__device__ __forceinline__ void dc_load_x(const __nv_bfloat16* X, int K, int T, int blk, int g, int j, uint4 (&x)[TT / 4]) {
-  const int t0 = min(g, T - 1);
-  const uint4* p0 = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(t0) * K + blk * 64 + 16 * j);
-  x[0] = __ldg(p0);
-  x[1] = __ldg(p0 + 1);
-  if constexpr (TT == 16) {
-    const int t1 = min(g + 8, T - 1);
-    const uint4* p1 = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(t1) * K + blk * 64 + 16 * j);
-    x[2] = __ldg(p1);
-    x[3] = __ldg(p1 + 1);
-  }
-}
 __device__ __forceinline__ uint32_t dc_word(const uint4& v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
-// m16n8k16 step s (of the 4 in a 64-element block) against B fragments (b0, b1); the X operand holds
-// elements 16 j + 4 s .. + 3 of token rows g (and g + 8): the same in-block order as the B fragments.
-template <int TT>
-__device__ __forceinline__ void dc_step(float (&d)[4], const uint4 (&x)[TT / 4], int s, uint32_t b0, uint32_t b1) {
-  const uint32_t a0 = dc_word(x[s >> 1], 2 * (s & 1)), a2 = dc_word(x[s >> 1], 2 * (s & 1) + 1);
-  uint32_t a1 = 0, a3 = 0;
-  if constexpr (TT == 16) {
-    a1 = dc_word(x[2 + (s >> 1)], 2 * (s & 1));
-    a3 = dc_word(x[2 + (s >> 1)], 2 * (s & 1) + 1);
-  }
-  dc_mma(d, a0, a1, a2, a3, b0, b1);
-}
 
-// The CTA's share: on a load axis where A unit a spans [4a, 4a + 4) and NF4 unit k sits at 4 na + k,
-// CTA c takes the units whose start lies in [c L / G, (c + 1) L / G), L = 4 na + nu.
-struct DcShare { int a0, na, u0, nu; };
-__device__ __forceinline__ DcShare dc_share(int cta, int G, int nu_all, int na_all) {
-  const int64_t L = static_cast<int64_t>(kDcALoad) * na_all + nu_all;
+// The CTA's share: on a load axis where A tile a spans [4a, 4a + 4) and NF4 tile k sits at 4 na + k,
+// CTA c takes the tiles whose start lies in [c L / G, (c + 1) L / G), L = 4 na + nt.
+struct DcShare { int a0, na, t0, nt; };
+__device__ __forceinline__ DcShare dc_share(int cta, int G, int nt_all, int na_all) {
+  const int64_t L = static_cast<int64_t>(kDcALoad) * na_all + nt_all;
   const int64_t lo = static_cast<int64_t>(cta) * L / G, hi = static_cast<int64_t>(cta + 1) * L / G;
   const int64_t abase = static_cast<int64_t>(kDcALoad) * na_all;
   auto clamp = [](int64_t v, int64_t hi_) { return static_cast<int>(v < 0 ? 0 : v > hi_ ? hi_ : v); };
   DcShare s;
   s.a0 = clamp((lo + kDcALoad - 1) / kDcALoad, na_all);
   s.na = clamp((hi + kDcALoad - 1) / kDcALoad, na_all) - s.a0;
-  s.u0 = clamp(lo - abase, nu_all);
-  s.nu = clamp(hi - abase, nu_all) - s.u0;
+  s.t0 = clamp(lo - abase, nt_all);
+  s.nt = clamp(hi - abase, nt_all) - s.t0;
   return s;
 }
-// Pass q of the CTA: A passes (up to 2 A units) first, then NF4 passes of near-equal size (up to 8).
+// Pass q of the CTA: one A tile per pass first, then NF4 passes of near-equal size (up to PT tiles).
 struct DcPass { bool isA; int cnt, first; };
 __device__ __forceinline__ DcPass dc_pass(const DcShare& sh, int npa, int npn, int q) {
   DcPass r;
   if (q < npa) {
     r.isA = true;
-    r.first = q * kDcAUnits;
-    r.cnt = min(kDcAUnits, sh.na - r.first);
+    r.first = q;
+    r.cnt = 1;
   } else {
-    const int k = q - npa, b = sh.nu / npn, e = sh.nu % npn;
+    const int k = q - npa, b = sh.nt / npn, e = sh.nt % npn;
     r.isA = false;
     r.cnt = b + (k < e ? 1 : 0);
     r.first = k * b + min(k, e);
@@ -194,86 +171,94 @@ __device__ __forceinline__ DcPass dc_pass(const DcShare& sh, int npa, int npn, i
   return r;
 }
 
+// Registers of one stage for one lane: code words (NF4: tile q's rows g and g + 8 in c[q]; A: 32 bytes
+// of row g in c[0], c[1] and of row g + 8 in c[2], c[3]) and X words (token g in x[0], x[1]; token
+// g + 8 in x[2], x[3]).
+template <int TT> struct DcRegs {
+  uint4 c[4];
+  uint4 x[TT / 4];
+};
+// The A fragments of one 64-element block when the operand is bf16 already (A or B rows): MMA step s
+// takes words 2 s and 2 s + 1 of the lane's 16 elements in rows g (c[0], c[1]) and g + 8 (c[2], c[3]).
 template <int TT>
-__global__ void __launch_bounds__(kDcThreads, 1)
-    nf4_decode_kernel(const __grid_constant__ DcMaps maps, const DecParams p, const CodebookArg cb) {
+__device__ __forceinline__ void dc_frag_bf16(const DcRegs<TT>& R, uint32_t (&a)[16]) {
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    a[4 * s] = dc_word(R.c[s >> 1], 2 * (s & 1));
+    a[4 * s + 1] = dc_word(R.c[2 + (s >> 1)], 2 * (s & 1));
+    a[4 * s + 2] = dc_word(R.c[s >> 1], 2 * (s & 1) + 1);
+    a[4 * s + 3] = dc_word(R.c[2 + (s >> 1)], 2 * (s & 1) + 1);
+  }
+}
+// One 64-element block: d (rows g, g + 8 x tokens 2 j, 2 j + 1; + 8 for the second token half) +=
+// A fragments x the lane's X words; MMA step s uses elements 16 j + 4 s .. + 3 of both operands.
+template <int TT>
+__device__ __forceinline__ void dc_block_mma(float (&d)[TT == 16 ? 8 : 4], const uint32_t (&a)[16],
+                                             const DcRegs<TT>& R) {
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const uint4& xv = R.x[s >> 1];
+    dc_mma(d[0], d[1], d[2], d[3], a[4 * s], a[4 * s + 1], a[4 * s + 2], a[4 * s + 3], dc_word(xv, 2 * (s & 1)),
+           dc_word(xv, 2 * (s & 1) + 1));
+    if constexpr (TT == 16) {
+      const uint4& xw = R.x[2 + (s >> 1)];
+      dc_mma(d[4], d[5], d[6], d[7], a[4 * s], a[4 * s + 1], a[4 * s + 2], a[4 * s + 3], dc_word(xw, 2 * (s & 1)),
+             dc_word(xw, 2 * (s & 1) + 1));
+    }
+  }
+}
+
+template <int TT>
+__global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecParams p, const CodebookArg cb) {
+  constexpr int PT = TT == 16 ? 2 : kDcMaxTiles;      // tiles per pass
+  constexpr int NACC = TT == 16 ? 8 : 4;
   extern __shared__ __align__(1024) uint8_t dc_smem[];
   uint8_t* dsm = dc_smem;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, cta = blockIdx.x;
-  uint64_t* full = reinterpret_cast<uint64_t*>(dsm + kDcOffBar);
-  uint64_t* empty = full + kDcStages;
-  uint64_t* sready = empty + kDcStages;
-  uint64_t* suready = sready + 2;
+  uint64_t* cready = reinterpret_cast<uint64_t*>(dsm + kDcOffBar);
+  uint64_t* cfree = cready + kDcCRing;
+  uint64_t* suready = cfree + kDcCRing;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(suready + 1);
 
-  const DcShare sh = dc_share(cta, G, p.units, p.aunits);
-  const int npa = (sh.na + kDcAUnits - 1) / kDcAUnits;
-  const int npn = p.u_only ? 0 : (sh.nu + kDcUnits - 1) / kDcUnits;
+  const DcShare sh = dc_share(cta, G, p.tiles, p.atiles);
+  const int npa = sh.na;
+  const int npn = p.u_only ? 0 : (sh.nt + PT - 1) / PT;
   const int spp = (p.nkb + kDcStageBlocks - 1) / kDcStageBlocks;      // stages per pass
-  const int nrb = p.RP / 64;                                           // 64-wide column boxes of B
-  const int ulora = 32 / nrb;                                          // units per adapter stage
   const int nmain = (npa + npn) * spp;
-  const int total = nmain + (p.u_only ? 0 : (sh.nu + ulora - 1) / ulora);
+  const int nfirst = npa * spp;                                        // stages before the first NF4 one
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kDcStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kDcWarps);
+    for (int s = 0; s < kDcCRing; ++s) {
+      mbar_init(&cready[s], 1);
+      mbar_init(&cfree[s], kDcWarps);
     }
-    mbar_init(&sready[0], 1);
-    mbar_init(&sready[1], 1);
     mbar_init(suready, 1);
-    *abort_flag = (smem_u32(dsm) & 1023u) != 0 ? 1 : 0;   // the swizzled boxes need 1 KB alignment
+    *abort_flag = 0;
     fence_barrier_init();
   }
   __syncthreads();
-  if (*abort_flag) {
-    if (threadIdx.x == 0) raise_status(kStatusTimeout);
-    return;
-  }
 
   if (warp == kDcWarps) {
-    // ================================ TMA + block constants ================================
-    if (total == 0) return;
-    if (lane == 0) tma_prefetch_desc(&maps.b);
-    auto issue = [&](int i) {                       // lane 0
-      const int slot = i % kDcStages;
-      uint8_t* sb = dsm + kDcOffRing + slot * kDcSlotBytes;
-      if (i < nmain) {
-        const int st = i % spp;
-        const DcPass ps = dc_pass(sh, npa, npn, i / spp);
-        // one box per stage: 16 blocks x the pass's rows (blocks past K read as zeros and still count)
-        if (ps.isA) {
-          mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(ps.cnt * kDcStageBlocks * 1024));
-          tma_load_3d(sb, &maps.a[ps.cnt - 1], &full[slot], 0, (sh.a0 + ps.first) * 8, st * kDcStageBlocks);
-        } else {
-          mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(ps.cnt * kDcStageBlocks * 256));
-          tma_load_3d(sb, &maps.c[ps.cnt - 1], &full[slot], 0, (sh.u0 + ps.first) * 8, st * kDcStageBlocks);
-        }
-      } else {
-        const int first = (i - nmain) * ulora, cntl = min(ulora, sh.nu - first);
-        mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(cntl * nrb * min(p.r, 64) * 16));
-        for (int u = 0; u < cntl; ++u)
-          for (int c = 0; c < nrb; ++c)
-            tma_load_2d(sb + (u * nrb + c) * 1024, &maps.b, &full[slot], c * 64, (sh.u0 + first + u) * 8);
-      }
-    };
-    // Block constants of an NF4 stage, rows lane and lane + 32 of its pass. The raw E4M3 bytes and group
-    // scales are loaded three stages ahead (a ring of three register sets), so decoding a stage never
-    // waits for memory.
+    // ============================== block constants of every NF4 stage ==============================
+    if (nmain == 0) return;
+    const int nnf = nmain - nfirst;
+    if (nnf == 0) return;
     const float mu = __ldg(p.mu);
+    // Rows lane and lane + 32 of the pass; the raw E4M3 bytes and group scales of NF4 stage k sit in ring
+    // entry k % 3, loaded three stages before they are decoded.
     struct Raw { uint32_t ew[2][4]; float sa[2], sz[2]; };
-    auto fetch = [&](int i, Raw& f) {
-      if (i >= nmain) return;
+    auto fetch = [&](int k, Raw& f) {
+      if (k >= nnf) return;
+      const int i = nfirst + k;
       const DcPass ps = dc_pass(sh, npa, npn, i / spp);
-      if (ps.isA) return;
       const int blk0 = (i % spp) * kDcStageBlocks, nbh = min(kDcStageBlocks, p.nkb - blk0);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int rho = lane + 32 * h;
-        if (rho < ps.cnt * 8) {
-          const int64_t e0 = static_cast<int64_t>((sh.u0 + ps.first) * 8 + rho) * p.nkb + blk0;
+        const int row = (sh.t0 + ps.first) * 16 + rho;
+        if (rho < ps.cnt * 16 && row < p.N) {
+          const int64_t e0 = static_cast<int64_t>(row) * p.nkb + blk0;
           const uint8_t* src = p.e4m3 + e0;
           if (nbh == 16 && (reinterpret_cast<uintptr_t>(src) & 15) == 0) {
             const uint4 v = __ldg(reinterpret_cast<const uint4*>(src));
@@ -296,71 +281,68 @@ __global__ void __launch_bounds__(kDcThreads, 1)
         }
       }
     };
-    Raw r0, r1, r2;
-    auto scales = [&](int i) {                      // whole warp; decodes r0 (stage i), then shifts the ring
-      const int cbi = i & 1;
-      if (i < nmain) {
-        const DcPass ps = dc_pass(sh, npa, npn, i / spp);
-        if (!ps.isA) {
-          const int blk0 = (i % spp) * kDcStageBlocks, nbh = min(kDcStageBlocks, p.nkb - blk0);
-          float* cbuf = reinterpret_cast<float*>(dsm + kDcOffCbuf + cbi * kDcCbufBytes);
+    // cbuf[block][tile][g] = (c1_hat of row g, of row g + 8) of the tile: what lane (g, j) of the consumer
+    // warp that takes the block multiplies its MMA results by
+    auto decode = [&](int k, const Raw& r) {
+      const int i = nfirst + k;
+      const DcPass ps = dc_pass(sh, npa, npn, i / spp);
+      const int blk0 = (i % spp) * kDcStageBlocks, nbh = min(kDcStageBlocks, p.nkb - blk0);
+      float* cbuf = reinterpret_cast<float*>(dsm + kDcOffCbuf + (k % kDcCRing) * kDcCbufBytes);
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int rho = lane + 32 * h;
-            if (rho < ps.cnt * 8) {
-              // the group of block b: g0 for b below the first group boundary in the stage, else the next
-              const int64_t e0 = static_cast<int64_t>((sh.u0 + ps.first) * 8 + rho) * p.nkb + blk0;
-              const int bsplit = static_cast<int>(256 - (e0 & 255));   // >= 1; >= 16: one group
-              float* dst = cbuf + ((rho & 7) >> 1) * (kDcUnits * 2) + (rho >> 3) * 2 + (rho & 1);
+      for (int h = 0; h < 2; ++h) {
+        const int rho = lane + 32 * h;
+        const int row = (sh.t0 + ps.first) * 16 + rho;
+        if (rho < ps.cnt * 16) {
+          const int64_t e0 = static_cast<int64_t>(row) * p.nkb + blk0;
+          const int bsplit = static_cast<int>(256 - (e0 & 255));   // blocks below it take the first scale
+          const bool valid = row < p.N;
+          float* dst = cbuf + ((rho >> 4) * 8 + (rho & 7)) * 2 + ((rho >> 3) & 1);
 #pragma unroll
-              for (int b = 0; b < 16; ++b) {
-                const float s2v = b < bsplit ? r0.sa[h] : r0.sz[h];
-                const uint8_t e = static_cast<uint8_t>(r0.ew[h][b >> 2] >> (8 * (b & 3)));
-                dst[b * (4 * kDcUnits * 2)] = b < nbh ? __fmaf_rn(decode_e4m3(e), s2v, mu) : 0.0f;
-              }
-            }
+          for (int b = 0; b < 16; b += 2) {               // two E4M3 values per conversion (exact in fp16)
+            const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
+                static_cast<__nv_fp8x2_storage_t>(r.ew[h][b >> 2] >> (8 * (b & 3))), __NV_E4M3);
+            const float2 dv = __half22float2(__half2(hr));
+            dst[b * (kDcMaxTiles * 16)] =
+                valid && b < nbh ? __fmaf_rn(dv.x, b < bsplit ? r.sa[h] : r.sz[h], mu) : 0.0f;
+            dst[(b + 1) * (kDcMaxTiles * 16)] =
+                valid && b + 1 < nbh ? __fmaf_rn(dv.y, b + 1 < bsplit ? r.sa[h] : r.sz[h], mu) : 0.0f;
           }
         }
       }
-      r0 = r1;
-      r1 = r2;
-      fetch(i + 3, r2);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sready[cbi]);
     };
-    if (lane == 0)
-      for (int i = 0; i < min(kDcStages, total); ++i) issue(i);
-    fetch(0, r0);
-    fetch(1, r1);
-    fetch(2, r2);
-    scales(0);
-    // Iteration i: the constants of stage i + 1 (their buffer last held stage i - 1's, released at
-    // iteration i - 1), then wait until every consumer warp is done with stage i and refill its slot.
-    int issued = min(kDcStages, total);
-    for (int i = 0; i < total; ++i) {
-      if (*abort_flag) break;
-      if (i + 1 < total) scales(i + 1);
-      if (lane == 0) {
-        if (!mbar_wait(&empty[i % kDcStages], static_cast<uint32_t>((i / kDcStages) & 1))) {
+    Raw ring[3];
+    fetch(0, ring[0]);
+    fetch(1, ring[1]);
+    fetch(2, ring[2]);
+    bool go = true;
+    for (int k0 = 0; k0 < nnf && go; k0 += 3) {
+#pragma unroll
+      for (int u = 0; u < 3; ++u) {
+        const int k = k0 + u;
+        if (k >= nnf) break;
+        // its buffer last held NF4 stage k - R: wait until every consumer warp has read it
+        if (k >= kDcCRing && lane == 0 &&
+            !mbar_wait(&cfree[k % kDcCRing], static_cast<uint32_t>(((k / kDcCRing) - 1) & 1)))
           *abort_flag = 1;
-        } else if (i + kDcStages < total) {
-          issue(i + kDcStages);
-          issued = i + kDcStages + 1;
+        __syncwarp();
+        if (*abort_flag) {
+          go = false;
+          break;
         }
+        decode(k, ring[u]);
+        fetch(k + 3, ring[u]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&cready[k % kDcCRing]);
       }
-      __syncwarp();
     }
-    if (lane == 0)                                  // every issued copy has landed before the CTA exits
-      for (int k = max(0, issued - kDcStages); k < issued; ++k)
-        mbar_wait_short(&full[k % kDcStages], static_cast<uint32_t>((k / kDcStages) & 1));
     return;
   }
 
   if (warp == kDcWarps + 1) {
-    // ==================== gather sU (every A unit's tag) into shared memory ====================
+    // ==================== gather sU (every A tile's tag) into shared memory ====================
     if (p.u_only) return;
     bool ok = true;
-    for (int a = 0; a < p.aunits && ok; ++a)
+    for (int a = 0; a < p.atiles && ok; ++a)
       if (!wait_word_eq(p.tags + a, p.seq)) ok = false;
     // [T][RP] bf16, columns past r zero; 16-byte pieces, four in flight per lane
     const int pieces = p.T * (p.RP / 8), per_row = p.RP / 8;
@@ -390,7 +372,7 @@ __global__ void __launch_bounds__(kDcThreads, 1)
   const int w = warp, g = lane >> 2, j = lane & 3;
   const uint32_t lanebyte = 4u * lane;
   const int T = p.T;
-  if (nmain == 0) return;                           // u_only and no A unit here: nothing to do
+  if (nmain == 0) return;                           // u_only and no A tile here: nothing to do
   // the lookup table: entry e = (level[e >> 4], level[e & 15]) as a bf16 pair, one copy per lane
   for (int i = threadIdx.x; i < 256 * 32; i += 32 * kDcWarps) {
     const int e = i >> 5;
@@ -398,170 +380,214 @@ __global__ void __launch_bounds__(kDcThreads, 1)
   }
   dc_bar_consumers();
 
-  float* base = p.base_in_smem ? reinterpret_cast<float*>(dsm + kDcOffBase)
-                               : p.base_ws + static_cast<int64_t>(sh.u0) * T * 8;   // [unit][T][8]
+  float* base = p.base_ws + static_cast<int64_t>(sh.t0) * 16 * T;   // [tile][16][T]
+  const uint32_t ring0 = kDcOffRing + w * kDcRing * kDcWarpSlot;
+  // Stage i's bytes of block w into this warp's slot i % R, one commit group per stage (empty past the end).
+  // NF4: tile q's 16 rows x 32 B at (16 q + row) * 32 (piece: lane = 2 row + half, one per tile). A: 16 rows
+  // x 128 B, 16-byte piece pp of row rho at rho * 128 + (pp ^ (rho & 7)) * 16 (four per lane). Pieces
+  // outside the matrix are zero-filled without a read.
+  auto issue = [&](int i) {
+    if (i < nmain) {
+      const int blk = (i % spp) * kDcStageBlocks + w;
+      const DcPass ps = dc_pass(sh, npa, npn, i / spp);
+      const uint32_t slot = smem_u32(dsm) + ring0 + (i % kDcRing) * kDcWarpSlot;
+      if (ps.isA) {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int pc = lane + 32 * m, rho = pc >> 3, pp = pc & 7;
+          const int row = (sh.a0 + ps.first) * 16 + rho;
+          const bool ok = blk < p.nkb && row < p.r;
+          const __nv_bfloat16* src = ok ? p.A + static_cast<int64_t>(row) * p.K + blk * 64 + 8 * pp : p.A;
+          dc_cp16(slot + rho * 128 + ((pp ^ (rho & 7)) << 4), src, ok ? 16u : 0u);
+        }
+      } else {
+        const int rho = lane >> 1, h = lane & 1;
+#pragma unroll
+        for (int q = 0; q < PT; ++q) {
+          const int row = (sh.t0 + ps.first + q) * 16 + rho;
+          const bool ok = q < ps.cnt && blk < p.nkb && row < p.N;
+          const uint8_t* src = ok ? p.codes + static_cast<int64_t>(row) * (p.K / 2) + blk * 32 + 16 * h : p.codes;
+          dc_cp16(slot + (q * 16 + rho) * 32 + 16 * h, src, ok ? 16u : 0u);
+        }
+      }
+    }
+    dc_cp_commit();
+  };
+  // stage i's X words of block w (zero where there are none)
+  auto loadx = [&](int i, DcRegs<TT>& R) {
+#pragma unroll
+    for (int q = 0; q < TT / 4; ++q) R.x[q] = make_uint4(0, 0, 0, 0);
+    if (i >= nmain) return;
+    const int blk = (i % spp) * kDcStageBlocks + w;
+    if (blk >= p.nkb) return;
+    const __nv_bfloat16* xp = p.X + blk * 64 + 16 * j;
+    if (g < T) {
+      R.x[0] = __ldg(reinterpret_cast<const uint4*>(xp + static_cast<int64_t>(g) * p.K));
+      R.x[1] = __ldg(reinterpret_cast<const uint4*>(xp + static_cast<int64_t>(g) * p.K + 8));
+    }
+    if constexpr (TT == 16) {
+      if (g + 8 < T) {
+        R.x[2] = __ldg(reinterpret_cast<const uint4*>(xp + static_cast<int64_t>(g + 8) * p.K));
+        R.x[3] = __ldg(reinterpret_cast<const uint4*>(xp + static_cast<int64_t>(g + 8) * p.K + 8));
+      }
+    }
+  };
+
+  float acc[PT][NACC];
   bool live = true;
-  int i = 0;                                        // global stage index
-  // X fragments for this warp's block column, PD stages ahead (a ring of register sets shifted each stage;
-  // X stays in L2, so its latency is that of an L2 hit)
-  constexpr int PD = TT == 16 ? 1 : 2;
-  uint4 xr[PD + 1][TT / 4];
-  auto xvalid = [&](int ii) { return ii < nmain && (ii % spp) * kDcStageBlocks + w < p.nkb; };
+  auto stage = [&](int i, DcRegs<TT>& R) {
+    const int st = i % spp;
+    const DcPass ps = dc_pass(sh, npa, npn, i / spp);
+    if (st == 0) {
 #pragma unroll
-  for (int k = 0; k < PD; ++k)
-    if (xvalid(k)) dc_load_x<TT>(p.X, p.K, T, (k % spp) * kDcStageBlocks + w, g, j, xr[k]);
-  for (int q = 0; q < npa + npn; ++q) {
-    const DcPass ps = dc_pass(sh, npa, npn, q);
-    float acc[kDcUnits][TT == 16 ? 4 : 2];
+      for (int q = 0; q < PT; ++q)
 #pragma unroll
-    for (int u = 0; u < kDcUnits; ++u)
-#pragma unroll
-      for (int c = 0; c < (TT == 16 ? 4 : 2); ++c) acc[u][c] = 0.0f;
-    for (int st = 0; st < spp; ++st, ++i) {
-      const int slot = i % kDcStages;
-      const int blk = st * kDcStageBlocks + w;
-      const bool has = blk < p.nkb;
-      if (xvalid(i + PD)) dc_load_x<TT>(p.X, p.K, T, ((i + PD) % spp) * kDcStageBlocks + w, g, j, xr[PD]);
-      const uint4 (&xa)[TT / 4] = xr[0];
-      if (live && *abort_flag) live = false;
-      if (live && !mbar_wait(&sready[i & 1], static_cast<uint32_t>((i >> 1) & 1))) live = false;
-      if (live && !mbar_wait(&full[slot], static_cast<uint32_t>((i / kDcStages) & 1))) live = false;
+        for (int c = 0; c < NACC; ++c) acc[q][c] = 0.0f;
+    }
+    const bool has = st * kDcStageBlocks + w < p.nkb;
+    const uint32_t slot = ring0 + (i % kDcRing) * kDcWarpSlot;
+    if (live && *abort_flag) live = false;
+    if (ps.isA) {
+      if (live && has) {                            // A rows are bf16 already: row g in c[0..1], g + 8 in c[2..3]
+        const uint32_t r0 = slot + g * 128, r1 = slot + (g + 8) * 128;
+        R.c[0] = dc_ld128(dsm, r0 + (((2 * j) ^ g) << 4));
+        R.c[1] = dc_ld128(dsm, r0 + (((2 * j + 1) ^ g) << 4));
+        R.c[2] = dc_ld128(dsm, r1 + (((2 * j) ^ g) << 4));
+        R.c[3] = dc_ld128(dsm, r1 + (((2 * j + 1) ^ g) << 4));
+        uint32_t a[16];
+        dc_frag_bf16<TT>(R, a);
+        dc_block_mma<TT>(acc[0], a, R);
+      }
+    } else {
+      const int k = i - nfirst, cslot = k % kDcCRing;
+      if (live && !mbar_wait(&cready[cslot], static_cast<uint32_t>((k / kDcCRing) & 1))) live = false;
       if (!live) *abort_flag = 1;
-      const uint32_t sbase = kDcOffRing + slot * kDcSlotBytes;
-      if (live && has && ps.isA) {
-        // bf16 rows of A: lane (g, j) reads elements 16 j .. 16 j + 15 of row g (chunks 2 j, 2 j + 1)
+      float2 cs[PT];
+      const uint32_t cbase = kDcOffCbuf + cslot * kDcCbufBytes + (w * kDcMaxTiles * 8 + g) * 8;
 #pragma unroll
-        for (int a = 0; a < kDcAUnits; ++a) {
-          if (a >= ps.cnt) break;
-          const uint32_t rb = sbase + (w * ps.cnt + a) * 1024 + g * 128;
-          const uint4 v0 = dc_ld128(dsm, rb + (((2 * j) ^ g) << 4)), v1 = dc_ld128(dsm, rb + (((2 * j + 1) ^ g) << 4));
-          float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-          dc_step<TT>(d, xa, 0, v0.x, v0.y);
-          dc_step<TT>(d, xa, 1, v0.z, v0.w);
-          dc_step<TT>(d, xa, 2, v1.x, v1.y);
-          dc_step<TT>(d, xa, 3, v1.z, v1.w);
-#pragma unroll
-          for (int c = 0; c < (TT == 16 ? 4 : 2); ++c) acc[a][c] += d[c];
-        }
-      } else if (live && has) {
-        const uint32_t sb = sbase + w * (ps.cnt * 256) + g * 32 + j * 8;
-        const uint32_t cs_base = kDcOffCbuf + (i & 1) * kDcCbufBytes + ((w * 4 + j) * kDcUnits) * 8;
-#pragma unroll
-        for (int u = 0; u < kDcUnits; u += 2) {
-          if (u >= ps.cnt) break;
-          const uint4 cs = dc_ld128(dsm, cs_base + u * 8);      // (unit u: rows 2j, 2j+1), (unit u+1: ...)
-#pragma unroll
-          for (int uu = 0; uu < 2; ++uu) {
-            if (u + uu >= ps.cnt) break;
-            const uint2 cw = dc_ld64(dsm, sb + (u + uu) * 256);
-            uint32_t b[8];
-            b[0] = dc_pair<0>(dsm, cw.x, lanebyte); b[1] = dc_pair<1>(dsm, cw.x, lanebyte);
-            b[2] = dc_pair<2>(dsm, cw.x, lanebyte); b[3] = dc_pair<3>(dsm, cw.x, lanebyte);
-            b[4] = dc_pair<0>(dsm, cw.y, lanebyte); b[5] = dc_pair<1>(dsm, cw.y, lanebyte);
-            b[6] = dc_pair<2>(dsm, cw.y, lanebyte); b[7] = dc_pair<3>(dsm, cw.y, lanebyte);
-            float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-            for (int s = 0; s < 4; ++s) dc_step<TT>(d, xa, s, b[2 * s], b[2 * s + 1]);
-            const float c0 = __uint_as_float(uu ? cs.z : cs.x), c1 = __uint_as_float(uu ? cs.w : cs.y);
-            acc[u + uu][0] = __fmaf_rn(c0, d[0], acc[u + uu][0]);
-            acc[u + uu][1] = __fmaf_rn(c1, d[1], acc[u + uu][1]);
-            if constexpr (TT == 16) {
-              acc[u + uu][2] = __fmaf_rn(c0, d[2], acc[u + uu][2]);
-              acc[u + uu][3] = __fmaf_rn(c1, d[3], acc[u + uu][3]);
-            }
-          }
-        }
-      }
+      for (int q = 0; q < PT; ++q) cs[q] = dc_ldf2(dsm, cbase + q * 64);
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);
+      if (lane == 0) mbar_arrive(&cfree[cslot]);
+      if (live && has) {
 #pragma unroll
-      for (int k = 0; k < PD; ++k)
+        for (int q = 0; q < PT; ++q) {
+          if (q >= ps.cnt) break;
+          // A fragments: a[4 s + 0..3] = (row g, elements 4 s, 4 s + 1), (row g + 8, same),
+          // (row g, 4 s + 2, 4 s + 3), (row g + 8, same) of this lane's 16; byte 2 s and 2 s + 1 of 8
+          const uint2 c0 = dc_ld64(dsm, slot + (q * 16 + g) * 32 + 8 * j);
+          const uint2 c1 = dc_ld64(dsm, slot + (q * 16 + g + 8) * 32 + 8 * j);
+          uint32_t a[16];
+          a[0] = dc_pair<0>(dsm, c0.x, lanebyte);  a[1] = dc_pair<0>(dsm, c1.x, lanebyte);
+          a[2] = dc_pair<1>(dsm, c0.x, lanebyte);  a[3] = dc_pair<1>(dsm, c1.x, lanebyte);
+          a[4] = dc_pair<2>(dsm, c0.x, lanebyte);  a[5] = dc_pair<2>(dsm, c1.x, lanebyte);
+          a[6] = dc_pair<3>(dsm, c0.x, lanebyte);  a[7] = dc_pair<3>(dsm, c1.x, lanebyte);
+          a[8] = dc_pair<0>(dsm, c0.y, lanebyte);  a[9] = dc_pair<0>(dsm, c1.y, lanebyte);
+          a[10] = dc_pair<1>(dsm, c0.y, lanebyte); a[11] = dc_pair<1>(dsm, c1.y, lanebyte);
+          a[12] = dc_pair<2>(dsm, c0.y, lanebyte); a[13] = dc_pair<2>(dsm, c1.y, lanebyte);
+          a[14] = dc_pair<3>(dsm, c0.y, lanebyte); a[15] = dc_pair<3>(dsm, c1.y, lanebyte);
+          float d[NACC];
 #pragma unroll
-        for (int m = 0; m < TT / 4; ++m) xr[k][m] = xr[k + 1][m];
-    }
-    // ---- end of pass: the 16 warps' partial sums, added in warp order; tokens in rounds of 8 ----
-    const int rows = ps.cnt * 8;
+          for (int c = 0; c < NACC; ++c) d[c] = 0.0f;
+          dc_block_mma<TT>(d, a, R);
 #pragma unroll
-    for (int half = 0; half < (TT == 16 ? 2 : 1); ++half) {
-      const int tr0 = 8 * half, tn = min(8, T - tr0);
-      if (tn <= 0) break;
-      if (g < tn) {
-#pragma unroll
-        for (int u = 0; u < kDcUnits; ++u) {
-          if (u >= ps.cnt) break;
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int idx = ((w * rows) + u * 8 + 2 * j + hh) * tn + g;
-            *dc_red(dsm, idx) = acc[u][2 * half + hh];
-          }
+          for (int c = 0; c < NACC; ++c) acc[q][c] = __fmaf_rn((c & 2) ? cs[q].y : cs[q].x, d[c], acc[q][c]);
         }
       }
-      dc_bar_consumers();
-      for (int o = threadIdx.x; o < rows * tn; o += 32 * kDcWarps) {
-        const int ro = o / tn, t = o % tn;
-        float sum = 0.0f;
-#pragma unroll
-        for (int ww = 0; ww < kDcWarps; ++ww) sum += *dc_red(dsm, (ww * rows + ro) * tn + t);
-        if (ps.isA)                                 // sU = bf16(s * X A^T), column 8 (unit) + row
-          p.U[static_cast<int64_t>(tr0 + t) * p.r + (sh.a0 + ps.first) * 8 + ro] = __float2bfloat16_rn(p.s * sum);
-        else
-          base[(static_cast<int64_t>(ps.first + ro / 8) * T + tr0 + t) * 8 + (ro & 7)] = sum;
-      }
-      dc_bar_consumers();
     }
-    if (ps.isA && threadIdx.x == 0) {               // this pass's piece of sU is complete and visible
+    if (st != spp - 1) return;
+    // ---- end of pass: the 16 warps' partial sums, added in warp order ----
+    const int rows = ps.cnt * 16, prow = 16 * PT;
+#pragma unroll
+    for (int q = 0; q < PT; ++q) {
+      if (q >= ps.cnt) break;
+#pragma unroll
+      for (int c = 0; c < NACC; ++c) {
+        // accumulator c = 4 th + 2 hh + e: row 16 q + g + 8 hh, token 2 j + e + 8 th
+        const int row = 16 * q + g + 8 * ((c >> 1) & 1), tok = 2 * j + (c & 1) + 8 * (c >> 2);
+        if (tok < T) *dc_red(dsm, (w * prow + row) * T + tok) = acc[q][c];
+      }
+    }
+    dc_bar_consumers();
+    for (int o = threadIdx.x; o < rows * T; o += 32 * kDcWarps) {
+      const int ro = o / T, t = o % T;
+      float sum = 0.0f;
+#pragma unroll
+      for (int ww = 0; ww < kDcWarps; ++ww) sum += *dc_red(dsm, (ww * prow + ro) * T + t);
+      if (ps.isA) {                                 // sU = bf16(s * X A^T): column = A row
+        const int arow = (sh.a0 + ps.first) * 16 + ro;
+        if (arow < p.r) p.U[static_cast<int64_t>(t) * p.r + arow] = __float2bfloat16_rn(p.s * sum);
+      } else {
+        base[(static_cast<int64_t>(ps.first) * 16 + ro) * T + t] = sum;
+      }
+    }
+    dc_bar_consumers();
+    if (ps.isA && threadIdx.x == 0) {               // this A tile's piece of sU is complete and visible
       __threadfence();
-      for (int a = 0; a < ps.cnt; ++a) st_release_u64(p.tags + sh.a0 + ps.first + a, p.seq);
+      st_release_u64(p.tags + sh.a0 + ps.first, p.seq);
     }
-  }
-  if (p.u_only) return;
-  // ---- adapter term and output: Y = bf16(base + sU B^T) per unit ----
-  const int nl = total - nmain;
-  const uint32_t su = kDcOffSU;
-  const int bw = min(p.r, 64) * 2;                  // bytes per row of a B column box
-  bool su_ok = live;
-  if (su_ok && !mbar_wait(suready, 0)) su_ok = false;
-  if (su_ok && *abort_flag) su_ok = false;
-  for (int l = 0; l < nl; ++l, ++i) {
-    const int slot = i % kDcStages;
-    if (su_ok && *abort_flag) su_ok = false;
-    bool ok = su_ok && mbar_wait(&sready[i & 1], static_cast<uint32_t>((i >> 1) & 1)) &&
-              mbar_wait(&full[slot], static_cast<uint32_t>((i / kDcStages) & 1));
-    if (!ok) {
-      su_ok = false;
-      *abort_flag = 1;
-    }
-    const int first = l * ulora, cntl = min(ulora, sh.nu - first);
-    const uint32_t sb = kDcOffRing + slot * kDcSlotBytes;
-    for (int uu = w; ok && uu < cntl; uu += kDcWarps) {
-      const int ul = first + uu;
-      float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      for (int rc = 0; rc < nrb; ++rc) {
-        const uint32_t bb = sb + (uu * nrb + rc) * 1024 + g * bw;
-        uint4 bv[2], av[TT / 4];
+  };
+
+  // the flat stage sequence: stage i + R - 1's copies issued, stage i's awaited and computed; X one ahead
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int off = 32 * j + 16 * hh;
-          bv[hh] = off < bw ? dc_ld128(dsm, bb + off) : make_uint4(0, 0, 0, 0);
-          av[hh] = dc_ld128(dsm, su + (min(g, T - 1) * p.RP + rc * 64 + 16 * j) * 2 + 16 * hh);
-          if constexpr (TT == 16) av[2 + hh] = dc_ld128(dsm, su + (min(g + 8, T - 1) * p.RP + rc * 64 + 16 * j) * 2 + 16 * hh);
-        }
-#pragma unroll
-        for (int s = 0; s < 4; ++s) dc_step<TT>(d, av, s, dc_word(bv[s >> 1], 2 * (s & 1)), dc_word(bv[s >> 1], 2 * (s & 1) + 1));
-      }
-      const int n = (sh.u0 + ul) * 8 + 2 * j;
-#pragma unroll
-      for (int half = 0; half < (TT == 16 ? 2 : 1); ++half) {
-        const int t = g + 8 * half;
-        if (t < T) {
-          const float2 bs = *reinterpret_cast<const float2*>(base + (static_cast<int64_t>(ul) * T + t) * 8 + 2 * j);
-          const __nv_bfloat162 y = __floats2bfloat162_rn(bs.x + d[2 * half], bs.y + d[2 * half + 1]);
-          *reinterpret_cast<__nv_bfloat162*>(p.Y + static_cast<int64_t>(t) * p.N + n) = y;
-        }
-      }
-    }
+  for (int i = 0; i < kDcRing - 1; ++i) issue(i);
+  DcRegs<TT> ra, rb;
+  loadx(0, ra);
+  auto step = [&](int i, DcRegs<TT>& cur, DcRegs<TT>& nxt) {
+    issue(i + kDcRing - 1);
+    loadx(i + 1, nxt);
+    dc_cp_wait<kDcRing - 1>();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[slot]);
+    stage(i, cur);
+    __syncwarp();                                   // slot i % R is refilled by the next step's issue
+  };
+  for (int i = 0; i < nmain; i += 2) {
+    step(i, ra, rb);
+    if (i + 1 >= nmain) break;
+    step(i + 1, rb, ra);
+  }
+  dc_cp_wait<0>();
+  if (p.u_only) {
+    if (!live) raise_status(kStatusTimeout);
+    return;
+  }
+  // ---- adapter term and output: Y = bf16(base + sU B^T), tile by tile across the warps ----
+  bool su_ok = live && mbar_wait(suready, 0) && !*abort_flag;
+  if (!su_ok) *abort_flag = 1;
+  for (int tl = w; su_ok && tl < sh.nt; tl += kDcWarps) {
+    float d[NACC];
+#pragma unroll
+    for (int c = 0; c < NACC; ++c) d[c] = 0.0f;
+    for (int rc = 0; rc < p.RP / 64; ++rc) {
+      DcRegs<TT> R;
+      const int e0 = rc * 64 + 16 * j;              // this lane's 16 adapter columns of the chunk
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int n = (sh.t0 + tl) * 16 + g + 8 * h;
+        const __nv_bfloat16* bp = p.B + static_cast<int64_t>(n) * p.r + e0;
+        R.c[2 * h] = (n < p.N && e0 < p.r) ? __ldg(reinterpret_cast<const uint4*>(bp)) : make_uint4(0, 0, 0, 0);
+        R.c[2 * h + 1] =
+            (n < p.N && e0 + 8 < p.r) ? __ldg(reinterpret_cast<const uint4*>(bp + 8)) : make_uint4(0, 0, 0, 0);
+      }
+      const uint32_t su = kDcOffSU + (min(g, T - 1) * p.RP + e0) * 2;
+      R.x[0] = dc_ld128(dsm, su);
+      R.x[1] = dc_ld128(dsm, su + 16);
+      if constexpr (TT == 16) {
+        const uint32_t su1 = kDcOffSU + (min(g + 8, T - 1) * p.RP + e0) * 2;
+        R.x[2] = dc_ld128(dsm, su1);
+        R.x[3] = dc_ld128(dsm, su1 + 16);
+      }
+      uint32_t a[16];
+      dc_frag_bf16<TT>(R, a);
+      dc_block_mma<TT>(d, a, R);
+    }
+#pragma unroll
+    for (int c = 0; c < NACC; ++c) {
+      const int rl = g + 8 * ((c >> 1) & 1), tok = 2 * j + (c & 1) + 8 * (c >> 2);
+      const int n = (sh.t0 + tl) * 16 + rl;
+      if (tok < T && n < p.N)
+        p.Y[static_cast<int64_t>(tok) * p.N + n] =
+            __float2bfloat16_rn(base[(static_cast<int64_t>(tl) * 16 + rl) * T + tok] + d[c]);
+    }
   }
   if (!live || !su_ok) raise_status(kStatusTimeout);
 }
