@@ -14,10 +14,12 @@
 //     tile weighs 4 NF4 tiles: bf16 against 4-bit); each CTA contracts its tiles over the whole K, so no
 //     partial sum crosses CTAs;
 //   * passes of up to 4 tiles (2 for more than 8 tokens), each a sequence of stages of 16 blocks (1024
-//     contraction elements); consumer warp w takes block w of every stage. Each warp streams its own bytes
-//     (block w of the pass's rows, 32-byte sectors used whole) into a private ring of 4 shared-memory slots
-//     with cp.async, three stages ahead, so ~96 KB per SM are in flight without holding registers, and no
-//     warp waits for another to refill a slot;
+//     contraction elements); consumer warp w takes block w of every stage. A stage (64 rows x 512 B of
+//     codes, or 16 A rows x 2 KB) comes into a ring of 4 shared-memory slots by cp.async three stages
+//     ahead, ~96 KB per SM in flight without holding registers: each warp copies 4 whole 512-byte row
+//     segments (contiguous runs, which HBM serves a quarter faster than 32-byte pieces of 64 rows), one
+//     named barrier per stage publishes the slot, and 16-byte pieces are XOR-swizzled by row so the
+//     fragment loads are free of bank conflicts;
 //   * mma.sync m16n8k16 with the weight as the 16-row A operand and X as the 8-token B operand. The A
 //     fragments come from code bytes: prmt forms (byte << 8 | lane * 4) and one shared-memory load fetches
 //     the bf16 pair (level[hi], level[lo]) from a 256-entry table replicated per lane (entries 256 B
@@ -49,15 +51,15 @@ constexpr int kDcThreads = 32 * (kDcWarps + 2);       // + constants warp + gath
 constexpr int kDcMaxTiles = 4;                        // NF4 tiles per pass (2 when T > 8)
 constexpr int kDcALoad = 4;                           // an A tile weighs as much as 4 NF4 tiles
 constexpr int kDcStageBlocks = kDcWarps;
-constexpr int kDcRing = 4;                            // code slots per consumer warp
-constexpr int kDcWarpSlot = 2048;                     // one stage of one warp: 64 rows x 32 B, or 16 A rows x 128 B
+constexpr int kDcRing = 4;                            // stage slots
+constexpr int kDcSlotBytes = 32 * 1024;               // one stage: 64 rows x 512 B, or 16 A rows x 2 KB
 constexpr int kDcCRing = 4;                           // constant buffers (stages) in flight
 constexpr int kDcMaxTokens = 16;
 constexpr int kDcMaxRank = 256;
 constexpr int kDcLutBytes = 256 * 256;                // entry e at e * 256: lane copies in bytes 0..127
 constexpr int kDcOffRing = kDcLutBytes;
 constexpr int kDcCbufBytes = kDcStageBlocks * kDcMaxTiles * 8 * 8;   // [block][tile][g] (row g, row g + 8)
-constexpr int kDcOffCbuf = kDcOffRing + kDcWarps * kDcRing * kDcWarpSlot;
+constexpr int kDcOffCbuf = kDcOffRing + kDcRing * kDcSlotBytes;
 constexpr int kDcOffSU = kDcOffCbuf + kDcCRing * kDcCbufBytes;
 constexpr int kDcSUBytes = kDcMaxTokens * kDcMaxRank * 2;
 constexpr int kDcOffBar = kDcOffSU + kDcSUBytes;
@@ -154,22 +156,40 @@ __device__ __forceinline__ DcShare dc_share(int cta, int G, int nt_all, int na_a
   s.nt = clamp(hi - abase, nt_all) - s.t0;
   return s;
 }
-// Pass q of the CTA: one A tile per pass first, then NF4 passes of near-equal size (up to PT tiles).
+// Pass q of the CTA: one A tile per pass first, then NF4 passes of near-equal size (up to PT tiles):
+// nb = nt / npn tiles each, the first ne = nt % npn passes one more.
 struct DcPass { bool isA; int cnt, first; };
-__device__ __forceinline__ DcPass dc_pass(const DcShare& sh, int npa, int npn, int q) {
+__device__ __forceinline__ DcPass dc_pass(int npa, int nb, int ne, int q) {
   DcPass r;
   if (q < npa) {
     r.isA = true;
     r.first = q;
     r.cnt = 1;
   } else {
-    const int k = q - npa, b = sh.nt / npn, e = sh.nt % npn;
+    const int k = q - npa;
     r.isA = false;
-    r.cnt = b + (k < e ? 1 : 0);
-    r.first = k * b + min(k, e);
+    r.cnt = nb + (k < ne ? 1 : 0);
+    r.first = k * nb + min(k, ne);
   }
   return r;
 }
+// Position in the CTA's flat stage sequence, advanced one stage at a time (no divisions per stage).
+struct DcCursor {
+  int i, q, st;
+  DcPass ps;
+  __device__ __forceinline__ void init(int npa, int nb, int ne) {
+    i = 0; q = 0; st = 0;
+    ps = dc_pass(npa, nb, ne, 0);
+  }
+  __device__ __forceinline__ void next(int spp, int npa, int nb, int ne) {
+    ++i;
+    if (++st == spp) {
+      st = 0;
+      ++q;
+      ps = dc_pass(npa, nb, ne, q);
+    }
+  }
+};
 
 // Registers of one stage for one lane: code words (NF4: tile q's rows g and g + 8 in c[q]; A: 32 bytes
 // of row g in c[0], c[1] and of row g + 8 in c[2], c[3]) and X words (token g in x[0], x[1]; token
@@ -226,6 +246,7 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
   const int npn = p.u_only ? 0 : (sh.nt + PT - 1) / PT;
   const int spp = (p.nkb + kDcStageBlocks - 1) / kDcStageBlocks;      // stages per pass
   const int nmain = (npa + npn) * spp;
+  const int pnb = npn ? sh.nt / npn : 0, pne = npn ? sh.nt % npn : 0;
   const int nfirst = npa * spp;                                        // stages before the first NF4 one
 
   if (threadIdx.x == 0) {
@@ -251,7 +272,7 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
     auto fetch = [&](int k, Raw& f) {
       if (k >= nnf) return;
       const int i = nfirst + k;
-      const DcPass ps = dc_pass(sh, npa, npn, i / spp);
+      const DcPass ps = dc_pass(npa, pnb, pne, i / spp);
       const int blk0 = (i % spp) * kDcStageBlocks, nbh = min(kDcStageBlocks, p.nkb - blk0);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -285,7 +306,7 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
     // warp that takes the block multiplies its MMA results by
     auto decode = [&](int k, const Raw& r) {
       const int i = nfirst + k;
-      const DcPass ps = dc_pass(sh, npa, npn, i / spp);
+      const DcPass ps = dc_pass(npa, pnb, pne, i / spp);
       const int blk0 = (i % spp) * kDcStageBlocks, nbh = min(kDcStageBlocks, p.nkb - blk0);
       float* cbuf = reinterpret_cast<float*>(dsm + kDcOffCbuf + (k % kDcCRing) * kDcCbufBytes);
 #pragma unroll
@@ -381,45 +402,42 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
   dc_bar_consumers();
 
   float* base = p.base_ws + static_cast<int64_t>(sh.t0) * 16 * T;   // [tile][16][T]
-  const uint32_t ring0 = kDcOffRing + w * kDcRing * kDcWarpSlot;
-  // Stage i's bytes of block w into this warp's slot i % R, one commit group per stage (empty past the end).
-  // NF4: tile q's 16 rows x 32 B at (16 q + row) * 32 (piece: lane = 2 row + half, one per tile). A: 16 rows
-  // x 128 B, 16-byte piece pp of row rho at rho * 128 + (pp ^ (rho & 7)) * 16 (four per lane). Pieces
-  // outside the matrix are zero-filled without a read.
-  auto issue = [&](int i) {
-    if (i < nmain) {
-      const int blk = (i % spp) * kDcStageBlocks + w;
-      const DcPass ps = dc_pass(sh, npa, npn, i / spp);
-      const uint32_t slot = smem_u32(dsm) + ring0 + (i % kDcRing) * kDcWarpSlot;
-      if (ps.isA) {
+  // Stage c's bytes into slot c.i % R, one commit group per stage (empty past the end); this warp's share:
+  // NF4 rows 4 w .. 4 w + 3 of the pass (512 B each, piece pc of row rho at rho * 512 + (pc ^ (rho & 7)) * 16),
+  // or A row w (2 KB, piece pc at w * 2048 + (pc ^ (w & 7)) * 16). Pieces outside the matrix are zero-filled
+  // without a read.
+  auto issue = [&](const DcCursor& c) {
+    if (c.i < nmain) {
+      const uint32_t slot = smem_u32(dsm) + kDcOffRing + (c.i % kDcRing) * kDcSlotBytes;
+      if (c.ps.isA) {
+        const int row = (sh.a0 + c.ps.first) * 16 + w;
+        const int64_t e0 = static_cast<int64_t>(row) * p.K + c.st * 1024;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-          const int pc = lane + 32 * m, rho = pc >> 3, pp = pc & 7;
-          const int row = (sh.a0 + ps.first) * 16 + rho;
-          const bool ok = blk < p.nkb && row < p.r;
-          const __nv_bfloat16* src = ok ? p.A + static_cast<int64_t>(row) * p.K + blk * 64 + 8 * pp : p.A;
-          dc_cp16(slot + rho * 128 + ((pp ^ (rho & 7)) << 4), src, ok ? 16u : 0u);
+          const int pc = lane + 32 * m;
+          const bool ok = row < p.r && c.st * 1024 + 8 * pc < p.K;
+          dc_cp16(slot + w * 2048 + ((pc ^ (w & 7)) << 4), ok ? p.A + e0 + 8 * pc : p.A, ok ? 16u : 0u);
         }
       } else {
-        const int rho = lane >> 1, h = lane & 1;
+        const int b0 = c.st * 512 + 16 * lane;
 #pragma unroll
-        for (int q = 0; q < PT; ++q) {
-          const int row = (sh.t0 + ps.first + q) * 16 + rho;
-          const bool ok = q < ps.cnt && blk < p.nkb && row < p.N;
-          const uint8_t* src = ok ? p.codes + static_cast<int64_t>(row) * (p.K / 2) + blk * 32 + 16 * h : p.codes;
-          dc_cp16(slot + (q * 16 + rho) * 32 + 16 * h, src, ok ? 16u : 0u);
+        for (int m = 0; m < 4; ++m) {
+          const int rho = 4 * w + m;
+          const int row = (sh.t0 + c.ps.first) * 16 + rho;
+          const bool ok = rho < c.ps.cnt * 16 && row < p.N && b0 < p.K / 2;
+          const uint8_t* src = ok ? p.codes + static_cast<int64_t>(row) * (p.K / 2) + b0 : p.codes;
+          dc_cp16(slot + rho * 512 + ((lane ^ (rho & 7)) << 4), src, ok ? 16u : 0u);
         }
       }
     }
     dc_cp_commit();
   };
-  // stage i's X words of block w (zero where there are none)
-  auto loadx = [&](int i, DcRegs<TT>& R) {
+  // stage c's X words of block w (zero where there are none)
+  auto loadx = [&](const DcCursor& c, DcRegs<TT>& R) {
 #pragma unroll
     for (int q = 0; q < TT / 4; ++q) R.x[q] = make_uint4(0, 0, 0, 0);
-    if (i >= nmain) return;
-    const int blk = (i % spp) * kDcStageBlocks + w;
-    if (blk >= p.nkb) return;
+    const int blk = c.st * kDcStageBlocks + w;
+    if (c.i >= nmain || blk >= p.nkb) return;
     const __nv_bfloat16* xp = p.X + blk * 64 + 16 * j;
     if (g < T) {
       R.x[0] = __ldg(reinterpret_cast<const uint4*>(xp + static_cast<int64_t>(g) * p.K));
@@ -435,31 +453,31 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
 
   float acc[PT][NACC];
   bool live = true;
-  auto stage = [&](int i, DcRegs<TT>& R) {
-    const int st = i % spp;
-    const DcPass ps = dc_pass(sh, npa, npn, i / spp);
-    if (st == 0) {
+  int knf = 0;                                      // NF4 stages computed so far (the constants ring index)
+  auto stage = [&](const DcCursor& c, DcRegs<TT>& R) {
+    const DcPass& ps = c.ps;
+    if (c.st == 0) {
 #pragma unroll
       for (int q = 0; q < PT; ++q)
 #pragma unroll
-        for (int c = 0; c < NACC; ++c) acc[q][c] = 0.0f;
+        for (int e = 0; e < NACC; ++e) acc[q][e] = 0.0f;
     }
-    const bool has = st * kDcStageBlocks + w < p.nkb;
-    const uint32_t slot = ring0 + (i % kDcRing) * kDcWarpSlot;
+    const bool has = c.st * kDcStageBlocks + w < p.nkb;
+    const uint32_t slot = kDcOffRing + (c.i % kDcRing) * kDcSlotBytes;
     if (live && *abort_flag) live = false;
     if (ps.isA) {
       if (live && has) {                            // A rows are bf16 already: row g in c[0..1], g + 8 in c[2..3]
-        const uint32_t r0 = slot + g * 128, r1 = slot + (g + 8) * 128;
-        R.c[0] = dc_ld128(dsm, r0 + (((2 * j) ^ g) << 4));
-        R.c[1] = dc_ld128(dsm, r0 + (((2 * j + 1) ^ g) << 4));
-        R.c[2] = dc_ld128(dsm, r1 + (((2 * j) ^ g) << 4));
-        R.c[3] = dc_ld128(dsm, r1 + (((2 * j + 1) ^ g) << 4));
+        const uint32_t r0 = slot + g * 2048, r1 = slot + (g + 8) * 2048;
+        R.c[0] = dc_ld128(dsm, r0 + (((8 * w + 2 * j) ^ g) << 4));
+        R.c[1] = dc_ld128(dsm, r0 + (((8 * w + 2 * j + 1) ^ g) << 4));
+        R.c[2] = dc_ld128(dsm, r1 + (((8 * w + 2 * j) ^ g) << 4));
+        R.c[3] = dc_ld128(dsm, r1 + (((8 * w + 2 * j + 1) ^ g) << 4));
         uint32_t a[16];
         dc_frag_bf16<TT>(R, a);
         dc_block_mma<TT>(acc[0], a, R);
       }
     } else {
-      const int k = i - nfirst, cslot = k % kDcCRing;
+      const int k = knf++, cslot = k % kDcCRing;
       if (live && !mbar_wait(&cready[cslot], static_cast<uint32_t>((k / kDcCRing) & 1))) live = false;
       if (!live) *abort_flag = 1;
       float2 cs[PT];
@@ -469,13 +487,15 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
       __syncwarp();
       if (lane == 0) mbar_arrive(&cfree[cslot]);
       if (live && has) {
+        // this lane's 8 bytes of block w in row rho: piece 2 w + j / 2 (swizzled), half j & 1
+        const uint32_t pof = ((((2 * w + (j >> 1)) ^ g) & 31) << 4) + 8 * (j & 1);
 #pragma unroll
         for (int q = 0; q < PT; ++q) {
           if (q >= ps.cnt) break;
           // A fragments: a[4 s + 0..3] = (row g, elements 4 s, 4 s + 1), (row g + 8, same),
           // (row g, 4 s + 2, 4 s + 3), (row g + 8, same) of this lane's 16; byte 2 s and 2 s + 1 of 8
-          const uint2 c0 = dc_ld64(dsm, slot + (q * 16 + g) * 32 + 8 * j);
-          const uint2 c1 = dc_ld64(dsm, slot + (q * 16 + g + 8) * 32 + 8 * j);
+          const uint2 c0 = dc_ld64(dsm, slot + (q * 16 + g) * 512 + pof);
+          const uint2 c1 = dc_ld64(dsm, slot + (q * 16 + g + 8) * 512 + pof);
           uint32_t a[16];
           a[0] = dc_pair<0>(dsm, c0.x, lanebyte);  a[1] = dc_pair<0>(dsm, c1.x, lanebyte);
           a[2] = dc_pair<1>(dsm, c0.x, lanebyte);  a[3] = dc_pair<1>(dsm, c1.x, lanebyte);
@@ -487,24 +507,24 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
           a[14] = dc_pair<3>(dsm, c0.y, lanebyte); a[15] = dc_pair<3>(dsm, c1.y, lanebyte);
           float d[NACC];
 #pragma unroll
-          for (int c = 0; c < NACC; ++c) d[c] = 0.0f;
+          for (int e = 0; e < NACC; ++e) d[e] = 0.0f;
           dc_block_mma<TT>(d, a, R);
 #pragma unroll
-          for (int c = 0; c < NACC; ++c) acc[q][c] = __fmaf_rn((c & 2) ? cs[q].y : cs[q].x, d[c], acc[q][c]);
+          for (int e = 0; e < NACC; ++e) acc[q][e] = __fmaf_rn((e & 2) ? cs[q].y : cs[q].x, d[e], acc[q][e]);
         }
       }
     }
-    if (st != spp - 1) return;
+    if (c.st != spp - 1) return;
     // ---- end of pass: the 16 warps' partial sums, added in warp order ----
     const int rows = ps.cnt * 16, prow = 16 * PT;
 #pragma unroll
     for (int q = 0; q < PT; ++q) {
       if (q >= ps.cnt) break;
 #pragma unroll
-      for (int c = 0; c < NACC; ++c) {
-        // accumulator c = 4 th + 2 hh + e: row 16 q + g + 8 hh, token 2 j + e + 8 th
-        const int row = 16 * q + g + 8 * ((c >> 1) & 1), tok = 2 * j + (c & 1) + 8 * (c >> 2);
-        if (tok < T) *dc_red(dsm, (w * prow + row) * T + tok) = acc[q][c];
+      for (int e = 0; e < NACC; ++e) {
+        // accumulator e = 4 th + 2 hh + u: row 16 q + g + 8 hh, token 2 j + u + 8 th
+        const int row = 16 * q + g + 8 * ((e >> 1) & 1), tok = 2 * j + (e & 1) + 8 * (e >> 2);
+        if (tok < T) *dc_red(dsm, (w * prow + row) * T + tok) = acc[q][e];
       }
     }
     dc_bar_consumers();
@@ -527,23 +547,35 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
     }
   };
 
-  // the flat stage sequence: stage i + R - 1's copies issued, stage i's awaited and computed; X one ahead
+  // The flat stage sequence. At stage i: wait for this thread's copies of stage i, then a barrier of the
+  // consumer warps (every warp's copies of stage i landed; every warp is done with stage i - 1, whose slot
+  // the copies of stage i + R - 1 reuse), issue those copies, load the next stage's X words, compute.
+  DcCursor cc, ci, cx;
+  cc.init(npa, pnb, pne);
+  ci.init(npa, pnb, pne);
 #pragma unroll
-  for (int i = 0; i < kDcRing - 1; ++i) issue(i);
+  for (int i = 0; i < kDcRing - 1; ++i) {
+    issue(ci);
+    ci.next(spp, npa, pnb, pne);
+  }
+  cx = cc;
   DcRegs<TT> ra, rb;
-  loadx(0, ra);
-  auto step = [&](int i, DcRegs<TT>& cur, DcRegs<TT>& nxt) {
-    issue(i + kDcRing - 1);
-    loadx(i + 1, nxt);
-    dc_cp_wait<kDcRing - 1>();
-    __syncwarp();
-    stage(i, cur);
-    __syncwarp();                                   // slot i % R is refilled by the next step's issue
+  loadx(cx, ra);
+  cx.next(spp, npa, pnb, pne);
+  auto step = [&](DcRegs<TT>& cur, DcRegs<TT>& nxt) {
+    dc_cp_wait<kDcRing - 2>();
+    dc_bar_consumers();
+    issue(ci);
+    ci.next(spp, npa, pnb, pne);
+    loadx(cx, nxt);
+    cx.next(spp, npa, pnb, pne);
+    stage(cc, cur);
+    cc.next(spp, npa, pnb, pne);
   };
-  for (int i = 0; i < nmain; i += 2) {
-    step(i, ra, rb);
-    if (i + 1 >= nmain) break;
-    step(i + 1, rb, ra);
+  while (cc.i < nmain) {
+    step(ra, rb);
+    if (cc.i >= nmain) break;
+    step(rb, ra);
   }
   dc_cp_wait<0>();
   if (p.u_only) {
