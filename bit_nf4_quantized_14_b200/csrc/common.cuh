@@ -63,13 +63,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// The same test, but a thread whose phase is not complete may be suspended (up to hint_ns) until it
+// completes: a waiting warp then takes no issue slots from the warps that compute beside it.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 // Wait for the phase with the given parity to complete. Returns false (and records a timeout in the
 // status word) if it has not completed within the wait limit in force (g_wait_limit_ns).
+constexpr uint32_t kSuspendHintNs = 20000;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns(), limit = *(volatile unsigned long long*)&g_wait_limit_ns;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_suspend(bar, parity, kSuspendHintNs)) return true;
     if (globaltimer_ns() - t0 > limit) {
       raise_status(kStatusTimeout);
       return false;
@@ -90,7 +104,7 @@ __device__ __forceinline__ bool wait_word_eq(const uint64_t* p, uint64_t want) {
   if (ld_acquire_u64(p) == want) return true;
   const unsigned long long t0 = globaltimer_ns(), limit = *(volatile unsigned long long*)&g_wait_limit_ns;
   while (true) {
-    __nanosleep(64);
+    __nanosleep(256);
     if (ld_acquire_u64(p) == want) return true;
     if (globaltimer_ns() - t0 > limit) {
       raise_status(kStatusTimeout);

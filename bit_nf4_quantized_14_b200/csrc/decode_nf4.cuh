@@ -26,8 +26,8 @@
 //     apart: no further arithmetic, no bank conflicts). Inside each 64-element block the MMA's k index is
 //     permuted (the same permutation on both operands) so lane j's 16 elements are 16 j .. 16 j + 15;
 //   * the block constant c1_hat = fma(decode(e4m3), s2, mu) multiplies the fp32 result of each block's four
-//     MMAs; a helper warp decodes each stage's constants into a ring of shared-memory buffers ahead of the
-//     consumers, from raw bytes it loads three stages ahead;
+//     MMAs; two helper warps (alternate stages) decode each stage's constants into a ring of shared-memory
+//     buffers ahead of the consumers, from raw bytes each loads three of its stages ahead;
 //   * at the end of each pass the 16 warps' partial sums meet in shared memory and are added in warp
 //     order (deterministic). A tiles come first: their sums, times s and rounded to bf16, are sU, which the
 //     CTA publishes with a per-call tag; a gather warp in every CTA waits for all of sU and copies it into
@@ -47,7 +47,8 @@
 namespace qnf4 {
 
 constexpr int kDcWarps = 16;                          // consumer warps: warp w takes block w of a stage
-constexpr int kDcThreads = 32 * (kDcWarps + 2);       // + constants warp + gather warp
+constexpr int kDcScaleWarps = 2;                      // constants warps, alternate NF4 stages
+constexpr int kDcThreads = 32 * (kDcWarps + kDcScaleWarps + 1);   // + constants warps + gather warp
 constexpr int kDcMaxTiles = 4;                        // NF4 tiles per pass (2 when T > 8)
 constexpr int kDcALoad = 4;                           // an A tile weighs as much as 4 NF4 tiles
 constexpr int kDcStageBlocks = kDcWarps;
@@ -56,15 +57,22 @@ constexpr int kDcSlotBytes = 32 * 1024;               // one stage: 64 rows x 51
 constexpr int kDcCRing = 4;                           // constant buffers (stages) in flight
 constexpr int kDcMaxTokens = 16;
 constexpr int kDcMaxRank = 256;
-constexpr int kDcLutBytes = 256 * 256;                // entry e at e * 256: lane copies in bytes 0..127
-constexpr int kDcOffRing = kDcLutBytes;
+// Shared memory. The lookup table (256 entries of 256 bytes, lane copies in bytes 0..127, the pass's partial
+// sums in bytes 128..255) sits at shared address 64 KB, so a byte permute forms a lookup's whole address
+// (0x1 << 16 | byte << 8 | lane * 4) with no add. Below it, from the dynamic base (a few KB at most): the
+// constant buffers, sU, the barriers and ring slot 0; above it, at 128 KB, ring slots 1..3.
+constexpr uint32_t kDcLutAddr = 1u << 16;
+constexpr uint32_t kDcHighAddr = 2u << 16;
 constexpr int kDcCbufBytes = kDcStageBlocks * kDcMaxTiles * 8 * 8;   // [block][tile][g] (row g, row g + 8)
-constexpr int kDcOffCbuf = kDcOffRing + kDcRing * kDcSlotBytes;
+constexpr int kDcOffCbuf = 0;
 constexpr int kDcOffSU = kDcOffCbuf + kDcCRing * kDcCbufBytes;
 constexpr int kDcSUBytes = kDcMaxTokens * kDcMaxRank * 2;
 constexpr int kDcOffBar = kDcOffSU + kDcSUBytes;
-constexpr int kDcSmemBytes = kDcOffBar + 128;
-static_assert(kDcSmemBytes <= 227 * 1024, "shared-memory budget");
+constexpr int kDcOffSlot0 = kDcOffBar + 1024;
+constexpr int kDcMaxBase = static_cast<int>(kDcLutAddr) - (kDcOffSlot0 + kDcSlotBytes);   // dynamic base limit
+constexpr int kDcSmemBytes = static_cast<int>(kDcHighAddr) + (kDcRing - 1) * kDcSlotBytes;  // enough for base 0
+static_assert(kDcMaxBase >= 4096 && kDcSmemBytes <= 227 * 1024, "shared-memory budget");
+static_assert(kDcCRing % kDcScaleWarps == 0, "each constants buffer belongs to one constants warp");
 
 struct DecParams {
   int T, N, K, r, RP;        // RP: r rounded up to 64
@@ -100,20 +108,29 @@ __device__ __forceinline__ uint32_t dc_prmt(uint32_t a, uint32_t b, uint32_t sel
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
   return d;
 }
-// Shared-memory loads as plain C++ loads from the __shared__ array (byte offsets from its start): the
-// compiler knows their address space and schedules them freely among the lookups and MMAs, and keeps
-// them after the mbarrier waits that publish the buffers (volatile asm with a memory clobber).
-__device__ __forceinline__ uint32_t dc_ld32(const uint8_t* sm, uint32_t off) {
-  return *reinterpret_cast<const uint32_t*>(sm + off);
+// Shared-memory loads by 32-bit shared address. Table lookups are plain asm (their addresses depend on
+// code bytes read after the barriers that publish the table and the stage, and the compiler may schedule
+// them freely); loads of ring slots and constant buffers are volatile, so they stay after the waits and
+// barriers that publish those buffers.
+__device__ __forceinline__ uint32_t dc_lut(uint32_t addr) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
 }
-__device__ __forceinline__ float2 dc_ldf2(const uint8_t* sm, uint32_t off) {
-  return *reinterpret_cast<const float2*>(sm + off);
+__device__ __forceinline__ uint2 dc_ld64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
 }
-__device__ __forceinline__ uint4 dc_ld128(const uint8_t* sm, uint32_t off) {
-  return *reinterpret_cast<const uint4*>(sm + off);
+__device__ __forceinline__ float2 dc_ldf2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
 }
-__device__ __forceinline__ uint2 dc_ld64(const uint8_t* sm, uint32_t off) {
-  return *reinterpret_cast<const uint2*>(sm + off);
+__device__ __forceinline__ uint4 dc_ld128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
 }
 // 16 bytes global -> shared through L2 only (cp.async.cg); src_bytes 0 writes 16 zero bytes and reads
 // nothing. Completion is tracked per thread in commit groups.
@@ -128,10 +145,11 @@ __device__ __forceinline__ void dc_cp_wait() {
 __device__ __forceinline__ void dc_bar_consumers() {   // the 16 consumer warps only
   asm volatile("bar.sync 1, %0;" ::"n"(32 * kDcWarps) : "memory");
 }
-// Byte k of w looked up in this lane's table copy: offset (w.byte_k << 8) | lane * 4 in one permute.
+// Byte k of w looked up in this lane's table copy: with lanebyte = 0x10000 | lane * 4, one permute gives
+// the address kDcLutAddr | (w.byte_k << 8) | lane * 4.
 template <int k>
-__device__ __forceinline__ uint32_t dc_pair(const uint8_t* sm, uint32_t w, uint32_t lanebyte) {
-  return dc_ld32(sm, dc_prmt(w, lanebyte, 0x5504u | (k << 4)));
+__device__ __forceinline__ uint32_t dc_pair(uint32_t w, uint32_t lanebyte) {
+  return dc_lut(dc_prmt(w, lanebyte, 0x7604u | (k << 4)));
 }
 // The fp32 partial-sum buffer of a pass lives in the free halves of the table's 256-byte entries.
 __device__ __forceinline__ float* dc_red(uint8_t* sm, int idx) {
@@ -255,13 +273,22 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
       mbar_init(&cfree[s], kDcWarps);
     }
     mbar_init(suready, 1);
-    *abort_flag = 0;
+    *abort_flag = smem_u32(dsm) > static_cast<uint32_t>(kDcMaxBase) ? 1 : 0;   // the layout needs a low base
     fence_barrier_init();
   }
   __syncthreads();
+  if (*abort_flag) {
+    if (threadIdx.x == 0) raise_status(kStatusTimeout);
+    return;
+  }
+  // shared address of ring slot s
+  auto slot_addr = [&](int s) -> uint32_t {
+    return s == 0 ? smem_u32(dsm) + kDcOffSlot0 : kDcHighAddr + static_cast<uint32_t>(s - 1) * kDcSlotBytes;
+  };
 
-  if (warp == kDcWarps) {
-    // ============================== block constants of every NF4 stage ==============================
+  if (warp >= kDcWarps && warp < kDcWarps + kDcScaleWarps) {
+    // ============== block constants of NF4 stages k = sw, sw + 2, ... (sw: this constants warp) ==============
+    const int sw = warp - kDcWarps;
     if (nmain == 0) return;
     const int nnf = nmain - nfirst;
     if (nnf == 0) return;
@@ -332,14 +359,14 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
       }
     };
     Raw ring[3];
-    fetch(0, ring[0]);
-    fetch(1, ring[1]);
-    fetch(2, ring[2]);
+    fetch(sw, ring[0]);
+    fetch(sw + kDcScaleWarps, ring[1]);
+    fetch(sw + 2 * kDcScaleWarps, ring[2]);
     bool go = true;
-    for (int k0 = 0; k0 < nnf && go; k0 += 3) {
+    for (int k0 = sw; k0 < nnf && go; k0 += 3 * kDcScaleWarps) {
 #pragma unroll
       for (int u = 0; u < 3; ++u) {
-        const int k = k0 + u;
+        const int k = k0 + u * kDcScaleWarps;
         if (k >= nnf) break;
         // its buffer last held NF4 stage k - R: wait until every consumer warp has read it
         if (k >= kDcCRing && lane == 0 &&
@@ -351,7 +378,7 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
           break;
         }
         decode(k, ring[u]);
-        fetch(k + 3, ring[u]);
+        fetch(k + 3 * kDcScaleWarps, ring[u]);
         __syncwarp();
         if (lane == 0) mbar_arrive(&cready[k % kDcCRing]);
       }
@@ -359,7 +386,7 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
     return;
   }
 
-  if (warp == kDcWarps + 1) {
+  if (warp == kDcWarps + kDcScaleWarps) {
     // ==================== gather sU (every A tile's tag) into shared memory ====================
     if (p.u_only) return;
     bool ok = true;
@@ -391,13 +418,15 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
 
   // ======================================== consumers ========================================
   const int w = warp, g = lane >> 2, j = lane & 3;
-  const uint32_t lanebyte = 4u * lane;
+  const uint32_t lanebyte = 0x10000u | (4u * lane);
+  const uint32_t sb = smem_u32(dsm);
+  uint8_t* lut = dsm + (kDcLutAddr - sb);            // generic pointer to the table
   const int T = p.T;
   if (nmain == 0) return;                           // u_only and no A tile here: nothing to do
   // the lookup table: entry e = (level[e >> 4], level[e & 15]) as a bf16 pair, one copy per lane
   for (int i = threadIdx.x; i < 256 * 32; i += 32 * kDcWarps) {
     const int e = i >> 5;
-    reinterpret_cast<uint32_t*>(dsm)[e * 64 + (i & 31)] = pack_bf16x2(cb.levels[e >> 4], cb.levels[e & 15]);
+    reinterpret_cast<uint32_t*>(lut)[e * 64 + (i & 31)] = pack_bf16x2(cb.levels[e >> 4], cb.levels[e & 15]);
   }
   dc_bar_consumers();
 
@@ -408,7 +437,7 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
   // without a read.
   auto issue = [&](const DcCursor& c) {
     if (c.i < nmain) {
-      const uint32_t slot = smem_u32(dsm) + kDcOffRing + (c.i % kDcRing) * kDcSlotBytes;
+      const uint32_t slot = slot_addr(c.i % kDcRing);
       if (c.ps.isA) {
         const int row = (sh.a0 + c.ps.first) * 16 + w;
         const int64_t e0 = static_cast<int64_t>(row) * p.K + c.st * 1024;
@@ -463,15 +492,15 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
         for (int e = 0; e < NACC; ++e) acc[q][e] = 0.0f;
     }
     const bool has = c.st * kDcStageBlocks + w < p.nkb;
-    const uint32_t slot = kDcOffRing + (c.i % kDcRing) * kDcSlotBytes;
+    const uint32_t slot = slot_addr(c.i % kDcRing);
     if (live && *abort_flag) live = false;
     if (ps.isA) {
       if (live && has) {                            // A rows are bf16 already: row g in c[0..1], g + 8 in c[2..3]
         const uint32_t r0 = slot + g * 2048, r1 = slot + (g + 8) * 2048;
-        R.c[0] = dc_ld128(dsm, r0 + (((8 * w + 2 * j) ^ g) << 4));
-        R.c[1] = dc_ld128(dsm, r0 + (((8 * w + 2 * j + 1) ^ g) << 4));
-        R.c[2] = dc_ld128(dsm, r1 + (((8 * w + 2 * j) ^ g) << 4));
-        R.c[3] = dc_ld128(dsm, r1 + (((8 * w + 2 * j + 1) ^ g) << 4));
+        R.c[0] = dc_ld128(r0 + (((8 * w + 2 * j) ^ g) << 4));
+        R.c[1] = dc_ld128(r0 + (((8 * w + 2 * j + 1) ^ g) << 4));
+        R.c[2] = dc_ld128(r1 + (((8 * w + 2 * j) ^ g) << 4));
+        R.c[3] = dc_ld128(r1 + (((8 * w + 2 * j + 1) ^ g) << 4));
         uint32_t a[16];
         dc_frag_bf16<TT>(R, a);
         dc_block_mma<TT>(acc[0], a, R);
@@ -483,7 +512,7 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
       float2 cs[PT];
       const uint32_t cbase = kDcOffCbuf + cslot * kDcCbufBytes + (w * kDcMaxTiles * 8 + g) * 8;
 #pragma unroll
-      for (int q = 0; q < PT; ++q) cs[q] = dc_ldf2(dsm, cbase + q * 64);
+      for (int q = 0; q < PT; ++q) cs[q] = dc_ldf2(sb + cbase + q * 64);
       __syncwarp();
       if (lane == 0) mbar_arrive(&cfree[cslot]);
       if (live && has) {
@@ -494,17 +523,17 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
           if (q >= ps.cnt) break;
           // A fragments: a[4 s + 0..3] = (row g, elements 4 s, 4 s + 1), (row g + 8, same),
           // (row g, 4 s + 2, 4 s + 3), (row g + 8, same) of this lane's 16; byte 2 s and 2 s + 1 of 8
-          const uint2 c0 = dc_ld64(dsm, slot + (q * 16 + g) * 512 + pof);
-          const uint2 c1 = dc_ld64(dsm, slot + (q * 16 + g + 8) * 512 + pof);
+          const uint2 c0 = dc_ld64(slot + (q * 16 + g) * 512 + pof);
+          const uint2 c1 = dc_ld64(slot + (q * 16 + g + 8) * 512 + pof);
           uint32_t a[16];
-          a[0] = dc_pair<0>(dsm, c0.x, lanebyte);  a[1] = dc_pair<0>(dsm, c1.x, lanebyte);
-          a[2] = dc_pair<1>(dsm, c0.x, lanebyte);  a[3] = dc_pair<1>(dsm, c1.x, lanebyte);
-          a[4] = dc_pair<2>(dsm, c0.x, lanebyte);  a[5] = dc_pair<2>(dsm, c1.x, lanebyte);
-          a[6] = dc_pair<3>(dsm, c0.x, lanebyte);  a[7] = dc_pair<3>(dsm, c1.x, lanebyte);
-          a[8] = dc_pair<0>(dsm, c0.y, lanebyte);  a[9] = dc_pair<0>(dsm, c1.y, lanebyte);
-          a[10] = dc_pair<1>(dsm, c0.y, lanebyte); a[11] = dc_pair<1>(dsm, c1.y, lanebyte);
-          a[12] = dc_pair<2>(dsm, c0.y, lanebyte); a[13] = dc_pair<2>(dsm, c1.y, lanebyte);
-          a[14] = dc_pair<3>(dsm, c0.y, lanebyte); a[15] = dc_pair<3>(dsm, c1.y, lanebyte);
+          a[0] = dc_pair<0>(c0.x, lanebyte);  a[1] = dc_pair<0>(c1.x, lanebyte);
+          a[2] = dc_pair<1>(c0.x, lanebyte);  a[3] = dc_pair<1>(c1.x, lanebyte);
+          a[4] = dc_pair<2>(c0.x, lanebyte);  a[5] = dc_pair<2>(c1.x, lanebyte);
+          a[6] = dc_pair<3>(c0.x, lanebyte);  a[7] = dc_pair<3>(c1.x, lanebyte);
+          a[8] = dc_pair<0>(c0.y, lanebyte);  a[9] = dc_pair<0>(c1.y, lanebyte);
+          a[10] = dc_pair<1>(c0.y, lanebyte); a[11] = dc_pair<1>(c1.y, lanebyte);
+          a[12] = dc_pair<2>(c0.y, lanebyte); a[13] = dc_pair<2>(c1.y, lanebyte);
+          a[14] = dc_pair<3>(c0.y, lanebyte); a[15] = dc_pair<3>(c1.y, lanebyte);
           float d[NACC];
 #pragma unroll
           for (int e = 0; e < NACC; ++e) d[e] = 0.0f;
@@ -524,7 +553,7 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
       for (int e = 0; e < NACC; ++e) {
         // accumulator e = 4 th + 2 hh + u: row 16 q + g + 8 hh, token 2 j + u + 8 th
         const int row = 16 * q + g + 8 * ((e >> 1) & 1), tok = 2 * j + (e & 1) + 8 * (e >> 2);
-        if (tok < T) *dc_red(dsm, (w * prow + row) * T + tok) = acc[q][e];
+        if (tok < T) *dc_red(lut, (w * prow + row) * T + tok) = acc[q][e];
       }
     }
     dc_bar_consumers();
@@ -532,7 +561,7 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
       const int ro = o / T, t = o % T;
       float sum = 0.0f;
 #pragma unroll
-      for (int ww = 0; ww < kDcWarps; ++ww) sum += *dc_red(dsm, (ww * prow + ro) * T + t);
+      for (int ww = 0; ww < kDcWarps; ++ww) sum += *dc_red(lut, (ww * prow + ro) * T + t);
       if (ps.isA) {                                 // sU = bf16(s * X A^T): column = A row
         const int arow = (sh.a0 + ps.first) * 16 + ro;
         if (arow < p.r) p.U[static_cast<int64_t>(t) * p.r + arow] = __float2bfloat16_rn(p.s * sum);
@@ -601,12 +630,12 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
             (n < p.N && e0 + 8 < p.r) ? __ldg(reinterpret_cast<const uint4*>(bp + 8)) : make_uint4(0, 0, 0, 0);
       }
       const uint32_t su = kDcOffSU + (min(g, T - 1) * p.RP + e0) * 2;
-      R.x[0] = dc_ld128(dsm, su);
-      R.x[1] = dc_ld128(dsm, su + 16);
+      R.x[0] = dc_ld128(sb + su);
+      R.x[1] = dc_ld128(sb + su + 16);
       if constexpr (TT == 16) {
         const uint32_t su1 = kDcOffSU + (min(g + 8, T - 1) * p.RP + e0) * 2;
-        R.x[2] = dc_ld128(dsm, su1);
-        R.x[3] = dc_ld128(dsm, su1 + 16);
+        R.x[2] = dc_ld128(sb + su1);
+        R.x[3] = dc_ld128(sb + su1 + 16);
       }
       uint32_t a[16];
       dc_frag_bf16<TT>(R, a);
