@@ -137,6 +137,9 @@ __device__ __forceinline__ uint4 dc_ld128(uint32_t addr) {
 __device__ __forceinline__ void dc_cp16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
+__device__ __forceinline__ void dc_cp16_full(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
 __device__ __forceinline__ void dc_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int kPending>
 __device__ __forceinline__ void dc_cp_wait() {
@@ -449,13 +452,22 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
         }
       } else {
         const int b0 = c.st * 512 + 16 * lane;
+        const int row0 = (sh.t0 + c.ps.first) * 16 + 4 * w;
+        if (4 * w + 3 < c.ps.cnt * 16 && row0 + 3 < p.N && c.st * 512 + 512 <= p.K / 2) {
+          // the common case: four whole row segments
+          const uint8_t* src = p.codes + static_cast<int64_t>(row0) * (p.K / 2) + b0;
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int rho = 4 * w + m;
-          const int row = (sh.t0 + c.ps.first) * 16 + rho;
-          const bool ok = rho < c.ps.cnt * 16 && row < p.N && b0 < p.K / 2;
-          const uint8_t* src = ok ? p.codes + static_cast<int64_t>(row) * (p.K / 2) + b0 : p.codes;
-          dc_cp16(slot + rho * 512 + ((lane ^ (rho & 7)) << 4), src, ok ? 16u : 0u);
+          for (int m = 0; m < 4; ++m)
+            dc_cp16_full(slot + (4 * w + m) * 512 + ((lane ^ ((4 * w + m) & 7)) << 4), src + m * (p.K / 2));
+        } else {
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int rho = 4 * w + m;
+            const int row = row0 + m;
+            const bool ok = rho < c.ps.cnt * 16 && row < p.N && b0 < p.K / 2;
+            const uint8_t* src = ok ? p.codes + static_cast<int64_t>(row) * (p.K / 2) + b0 : p.codes;
+            dc_cp16(slot + rho * 512 + ((lane ^ (rho & 7)) << 4), src, ok ? 16u : 0u);
+          }
         }
       }
     }
