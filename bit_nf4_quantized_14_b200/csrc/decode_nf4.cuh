@@ -46,12 +46,15 @@
 
 namespace qnf4 {
 
-constexpr int kDcWarps = 16;                          // consumer warps: warp w takes block w of a stage
+constexpr int kDcWarps = 8;                           // consumer warps: warp w takes blocks 2 w, 2 w + 1 of a stage
 constexpr int kDcScaleWarps = 2;                      // constants warps, alternate NF4 stages
 constexpr int kDcThreads = 32 * (kDcWarps + kDcScaleWarps + 1);   // + constants warps + gather warp
 constexpr int kDcMaxTiles = 4;                        // NF4 tiles per pass (2 when T > 8)
 constexpr int kDcALoad = 4;                           // an A tile weighs as much as 4 NF4 tiles
-constexpr int kDcStageBlocks = kDcWarps;
+constexpr int kDcStageBlocks = 16;
+constexpr int kDcBpw = kDcStageBlocks / kDcWarps;     // blocks per consumer warp and stage
+constexpr int kDcRowsPw = 64 / kDcWarps;              // NF4 rows each warp copies per stage
+constexpr int kDcARowsPw = 16 / kDcWarps;             // A rows each warp copies per stage
 constexpr int kDcRing = 4;                            // stage slots
 constexpr int kDcSlotBytes = 32 * 1024;               // one stage: 64 rows x 512 B, or 16 A rows x 2 KB
 constexpr int kDcCRing = 4;                           // constant buffers (stages) in flight
@@ -217,32 +220,31 @@ struct DcCursor {
 // g + 8 in x[2], x[3]).
 template <int TT> struct DcRegs {
   uint4 c[4];
-  uint4 x[TT / 4];
+  uint4 x[kDcBpw][TT / 4];
 };
 // The A fragments of one 64-element block when the operand is bf16 already (A or B rows): MMA step s
 // takes words 2 s and 2 s + 1 of the lane's 16 elements in rows g (c[0], c[1]) and g + 8 (c[2], c[3]).
-template <int TT>
-__device__ __forceinline__ void dc_frag_bf16(const DcRegs<TT>& R, uint32_t (&a)[16]) {
+__device__ __forceinline__ void dc_frag_bf16(const uint4 (&c)[4], uint32_t (&a)[16]) {
 #pragma unroll
   for (int s = 0; s < 4; ++s) {
-    a[4 * s] = dc_word(R.c[s >> 1], 2 * (s & 1));
-    a[4 * s + 1] = dc_word(R.c[2 + (s >> 1)], 2 * (s & 1));
-    a[4 * s + 2] = dc_word(R.c[s >> 1], 2 * (s & 1) + 1);
-    a[4 * s + 3] = dc_word(R.c[2 + (s >> 1)], 2 * (s & 1) + 1);
+    a[4 * s] = dc_word(c[s >> 1], 2 * (s & 1));
+    a[4 * s + 1] = dc_word(c[2 + (s >> 1)], 2 * (s & 1));
+    a[4 * s + 2] = dc_word(c[s >> 1], 2 * (s & 1) + 1);
+    a[4 * s + 3] = dc_word(c[2 + (s >> 1)], 2 * (s & 1) + 1);
   }
 }
 // One 64-element block: d (rows g, g + 8 x tokens 2 j, 2 j + 1; + 8 for the second token half) +=
 // A fragments x the lane's X words; MMA step s uses elements 16 j + 4 s .. + 3 of both operands.
 template <int TT>
 __device__ __forceinline__ void dc_block_mma(float (&d)[TT == 16 ? 8 : 4], const uint32_t (&a)[16],
-                                             const DcRegs<TT>& R) {
+                                             const uint4 (&x)[TT / 4]) {
 #pragma unroll
   for (int s = 0; s < 4; ++s) {
-    const uint4& xv = R.x[s >> 1];
+    const uint4& xv = x[s >> 1];
     dc_mma(d[0], d[1], d[2], d[3], a[4 * s], a[4 * s + 1], a[4 * s + 2], a[4 * s + 3], dc_word(xv, 2 * (s & 1)),
            dc_word(xv, 2 * (s & 1) + 1));
     if constexpr (TT == 16) {
-      const uint4& xw = R.x[2 + (s >> 1)];
+      const uint4& xw = x[2 + (s >> 1)];
       dc_mma(d[4], d[5], d[6], d[7], a[4 * s], a[4 * s + 1], a[4 * s + 2], a[4 * s + 3], dc_word(xw, 2 * (s & 1)),
              dc_word(xw, 2 * (s & 1) + 1));
     }
@@ -442,27 +444,32 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
     if (c.i < nmain) {
       const uint32_t slot = slot_addr(c.i % kDcRing);
       if (c.ps.isA) {
-        const int row = (sh.a0 + c.ps.first) * 16 + w;
-        const int64_t e0 = static_cast<int64_t>(row) * p.K + c.st * 1024;
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int pc = lane + 32 * m;
-          const bool ok = row < p.r && c.st * 1024 + 8 * pc < p.K;
-          dc_cp16(slot + w * 2048 + ((pc ^ (w & 7)) << 4), ok ? p.A + e0 + 8 * pc : p.A, ok ? 16u : 0u);
+        for (int ra = 0; ra < kDcARowsPw; ++ra) {
+          const int rho = kDcARowsPw * w + ra;
+          const int row = (sh.a0 + c.ps.first) * 16 + rho;
+          const int64_t e0 = static_cast<int64_t>(row) * p.K + c.st * 1024;
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int pc = lane + 32 * m;
+            const bool ok = row < p.r && c.st * 1024 + 8 * pc < p.K;
+            dc_cp16(slot + rho * 2048 + ((pc ^ (rho & 7)) << 4), ok ? p.A + e0 + 8 * pc : p.A, ok ? 16u : 0u);
+          }
         }
       } else {
         const int b0 = c.st * 512 + 16 * lane;
-        const int row0 = (sh.t0 + c.ps.first) * 16 + 4 * w;
-        if (4 * w + 3 < c.ps.cnt * 16 && row0 + 3 < p.N && c.st * 512 + 512 <= p.K / 2) {
-          // the common case: four whole row segments
+        const int rho0 = kDcRowsPw * w;
+        const int row0 = (sh.t0 + c.ps.first) * 16 + rho0;
+        if (rho0 + kDcRowsPw <= c.ps.cnt * 16 && row0 + kDcRowsPw <= p.N && c.st * 512 + 512 <= p.K / 2) {
+          // the common case: whole row segments
           const uint8_t* src = p.codes + static_cast<int64_t>(row0) * (p.K / 2) + b0;
 #pragma unroll
-          for (int m = 0; m < 4; ++m)
-            dc_cp16_full(slot + (4 * w + m) * 512 + ((lane ^ ((4 * w + m) & 7)) << 4), src + m * (p.K / 2));
+          for (int m = 0; m < kDcRowsPw; ++m)
+            dc_cp16_full(slot + (rho0 + m) * 512 + ((lane ^ ((rho0 + m) & 7)) << 4), src + m * (p.K / 2));
         } else {
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const int rho = 4 * w + m;
+          for (int m = 0; m < kDcRowsPw; ++m) {
+            const int rho = rho0 + m;
             const int row = row0 + m;
             const bool ok = rho < c.ps.cnt * 16 && row < p.N && b0 < p.K / 2;
             const uint8_t* src = ok ? p.codes + static_cast<int64_t>(row) * (p.K / 2) + b0 : p.codes;
@@ -473,21 +480,24 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
     }
     dc_cp_commit();
   };
-  // stage c's X words of block w (zero where there are none)
+  // stage c's X words of blocks kDcBpw w + b (zero where there are none)
   auto loadx = [&](const DcCursor& c, DcRegs<TT>& R) {
 #pragma unroll
-    for (int q = 0; q < TT / 4; ++q) R.x[q] = make_uint4(0, 0, 0, 0);
-    const int blk = c.st * kDcStageBlocks + w;
-    if (c.i >= nmain || blk >= p.nkb) return;
-    const __nv_bfloat16* xp = p.X + blk * 64 + 16 * j;
-    if (g < T) {
-      R.x[0] = __ldg(reinterpret_cast<const uint4*>(xp + static_cast<int64_t>(g) * p.K));
-      R.x[1] = __ldg(reinterpret_cast<const uint4*>(xp + static_cast<int64_t>(g) * p.K + 8));
-    }
-    if constexpr (TT == 16) {
-      if (g + 8 < T) {
-        R.x[2] = __ldg(reinterpret_cast<const uint4*>(xp + static_cast<int64_t>(g + 8) * p.K));
-        R.x[3] = __ldg(reinterpret_cast<const uint4*>(xp + static_cast<int64_t>(g + 8) * p.K + 8));
+    for (int b = 0; b < kDcBpw; ++b) {
+#pragma unroll
+      for (int q = 0; q < TT / 4; ++q) R.x[b][q] = make_uint4(0, 0, 0, 0);
+      const int blk = c.st * kDcStageBlocks + kDcBpw * w + b;
+      if (c.i >= nmain || blk >= p.nkb) continue;
+      const __nv_bfloat16* xp = p.X + blk * 64 + 16 * j;
+      if (g < T) {
+        R.x[b][0] = __ldg(reinterpret_cast<const uint4*>(xp + static_cast<int64_t>(g) * p.K));
+        R.x[b][1] = __ldg(reinterpret_cast<const uint4*>(xp + static_cast<int64_t>(g) * p.K + 8));
+      }
+      if constexpr (TT == 16) {
+        if (g + 8 < T) {
+          R.x[b][2] = __ldg(reinterpret_cast<const uint4*>(xp + static_cast<int64_t>(g + 8) * p.K));
+          R.x[b][3] = __ldg(reinterpret_cast<const uint4*>(xp + static_cast<int64_t>(g + 8) * p.K + 8));
+        }
       }
     }
   };
@@ -503,55 +513,69 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
 #pragma unroll
         for (int e = 0; e < NACC; ++e) acc[q][e] = 0.0f;
     }
-    const bool has = c.st * kDcStageBlocks + w < p.nkb;
     const uint32_t slot = slot_addr(c.i % kDcRing);
     if (live && *abort_flag) live = false;
     if (ps.isA) {
-      if (live && has) {                            // A rows are bf16 already: row g in c[0..1], g + 8 in c[2..3]
+#pragma unroll
+      for (int b = 0; b < kDcBpw; ++b) {
+        const int bw = kDcBpw * w + b;              // block of the stage
+        if (!live || c.st * kDcStageBlocks + bw >= p.nkb) continue;
+        // A rows are bf16 already: row g in c[0..1], g + 8 in c[2..3]
         const uint32_t r0 = slot + g * 2048, r1 = slot + (g + 8) * 2048;
-        R.c[0] = dc_ld128(r0 + (((8 * w + 2 * j) ^ g) << 4));
-        R.c[1] = dc_ld128(r0 + (((8 * w + 2 * j + 1) ^ g) << 4));
-        R.c[2] = dc_ld128(r1 + (((8 * w + 2 * j) ^ g) << 4));
-        R.c[3] = dc_ld128(r1 + (((8 * w + 2 * j + 1) ^ g) << 4));
+        R.c[0] = dc_ld128(r0 + (((8 * bw + 2 * j) ^ g) << 4));
+        R.c[1] = dc_ld128(r0 + (((8 * bw + 2 * j + 1) ^ g) << 4));
+        R.c[2] = dc_ld128(r1 + (((8 * bw + 2 * j) ^ g) << 4));
+        R.c[3] = dc_ld128(r1 + (((8 * bw + 2 * j + 1) ^ g) << 4));
         uint32_t a[16];
-        dc_frag_bf16<TT>(R, a);
-        dc_block_mma<TT>(acc[0], a, R);
+        dc_frag_bf16(R.c, a);
+        dc_block_mma<TT>(acc[0], a, R.x[b]);
       }
     } else {
       const int k = knf++, cslot = k % kDcCRing;
       if (live && !mbar_wait(&cready[cslot], static_cast<uint32_t>((k / kDcCRing) & 1))) live = false;
       if (!live) *abort_flag = 1;
-      float2 cs[PT];
-      const uint32_t cbase = kDcOffCbuf + cslot * kDcCbufBytes + (w * kDcMaxTiles * 8 + g) * 8;
+      float2 cs[kDcBpw][PT];
 #pragma unroll
-      for (int q = 0; q < PT; ++q) cs[q] = dc_ldf2(sb + cbase + q * 64);
+      for (int b = 0; b < kDcBpw; ++b) {
+        const uint32_t cbase = kDcOffCbuf + cslot * kDcCbufBytes + ((kDcBpw * w + b) * kDcMaxTiles * 8 + g) * 8;
+#pragma unroll
+        for (int q = 0; q < PT; ++q) cs[b][q] = dc_ldf2(sb + cbase + q * 64);
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&cfree[cslot]);
-      if (live && has) {
-        // this lane's 8 bytes of block w in row rho: piece 2 w + j / 2 (swizzled), half j & 1
-        const uint32_t pof = ((((2 * w + (j >> 1)) ^ g) & 31) << 4) + 8 * (j & 1);
+      // Tiles outer, blocks inner: the kDcBpw blocks of a tile are independent chains the scheduler can
+      // interleave. Blocks past K need no test: their constants are 0 and their X words 0, and the stale codes
+      // of their slot bytes only ever look up finite levels.
+      if (live) {
 #pragma unroll
         for (int q = 0; q < PT; ++q) {
           if (q >= ps.cnt) break;
-          // A fragments: a[4 s + 0..3] = (row g, elements 4 s, 4 s + 1), (row g + 8, same),
-          // (row g, 4 s + 2, 4 s + 3), (row g + 8, same) of this lane's 16; byte 2 s and 2 s + 1 of 8
-          const uint2 c0 = dc_ld64(slot + (q * 16 + g) * 512 + pof);
-          const uint2 c1 = dc_ld64(slot + (q * 16 + g + 8) * 512 + pof);
-          uint32_t a[16];
-          a[0] = dc_pair<0>(c0.x, lanebyte);  a[1] = dc_pair<0>(c1.x, lanebyte);
-          a[2] = dc_pair<1>(c0.x, lanebyte);  a[3] = dc_pair<1>(c1.x, lanebyte);
-          a[4] = dc_pair<2>(c0.x, lanebyte);  a[5] = dc_pair<2>(c1.x, lanebyte);
-          a[6] = dc_pair<3>(c0.x, lanebyte);  a[7] = dc_pair<3>(c1.x, lanebyte);
-          a[8] = dc_pair<0>(c0.y, lanebyte);  a[9] = dc_pair<0>(c1.y, lanebyte);
-          a[10] = dc_pair<1>(c0.y, lanebyte); a[11] = dc_pair<1>(c1.y, lanebyte);
-          a[12] = dc_pair<2>(c0.y, lanebyte); a[13] = dc_pair<2>(c1.y, lanebyte);
-          a[14] = dc_pair<3>(c0.y, lanebyte); a[15] = dc_pair<3>(c1.y, lanebyte);
-          float d[NACC];
 #pragma unroll
-          for (int e = 0; e < NACC; ++e) d[e] = 0.0f;
-          dc_block_mma<TT>(d, a, R);
+          for (int b = 0; b < kDcBpw; ++b) {
+            const int bw = kDcBpw * w + b;
+            // this lane's 8 bytes of block bw in rows g and g + 8 of tile q: piece 2 bw + j / 2 (swizzled), half j & 1
+            const uint32_t pof = ((((2 * bw + (j >> 1)) ^ g) & 31) << 4) + 8 * (j & 1);
+            const uint2 c0 = dc_ld64(slot + (q * 16 + g) * 512 + pof);
+            const uint2 c1 = dc_ld64(slot + (q * 16 + g + 8) * 512 + pof);
+            // A fragments: a[4 s + 0..3] = (row g, elements 4 s, 4 s + 1), (row g + 8, same),
+            // (row g, 4 s + 2, 4 s + 3), (row g + 8, same) of this lane's 16; byte 2 s and 2 s + 1 of 8
+            uint32_t a[16];
+            a[0] = dc_pair<0>(c0.x, lanebyte);  a[1] = dc_pair<0>(c1.x, lanebyte);
+            a[2] = dc_pair<1>(c0.x, lanebyte);  a[3] = dc_pair<1>(c1.x, lanebyte);
+            a[4] = dc_pair<2>(c0.x, lanebyte);  a[5] = dc_pair<2>(c1.x, lanebyte);
+            a[6] = dc_pair<3>(c0.x, lanebyte);  a[7] = dc_pair<3>(c1.x, lanebyte);
+            a[8] = dc_pair<0>(c0.y, lanebyte);  a[9] = dc_pair<0>(c1.y, lanebyte);
+            a[10] = dc_pair<1>(c0.y, lanebyte); a[11] = dc_pair<1>(c1.y, lanebyte);
+            a[12] = dc_pair<2>(c0.y, lanebyte); a[13] = dc_pair<2>(c1.y, lanebyte);
+            a[14] = dc_pair<3>(c0.y, lanebyte); a[15] = dc_pair<3>(c1.y, lanebyte);
+            float d[NACC];
 #pragma unroll
-          for (int e = 0; e < NACC; ++e) acc[q][e] = __fmaf_rn((e & 2) ? cs[q].y : cs[q].x, d[e], acc[q][e]);
+            for (int e = 0; e < NACC; ++e) d[e] = 0.0f;
+            dc_block_mma<TT>(d, a, R.x[b]);
+#pragma unroll
+            for (int e = 0; e < NACC; ++e)
+              acc[q][e] = __fmaf_rn((e & 2) ? cs[b][q].y : cs[b][q].x, d[e], acc[q][e]);
+          }
         }
       }
     }
@@ -642,16 +666,16 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
             (n < p.N && e0 + 8 < p.r) ? __ldg(reinterpret_cast<const uint4*>(bp + 8)) : make_uint4(0, 0, 0, 0);
       }
       const uint32_t su = kDcOffSU + (min(g, T - 1) * p.RP + e0) * 2;
-      R.x[0] = dc_ld128(sb + su);
-      R.x[1] = dc_ld128(sb + su + 16);
+      R.x[0][0] = dc_ld128(sb + su);
+      R.x[0][1] = dc_ld128(sb + su + 16);
       if constexpr (TT == 16) {
         const uint32_t su1 = kDcOffSU + (min(g + 8, T - 1) * p.RP + e0) * 2;
-        R.x[2] = dc_ld128(sb + su1);
-        R.x[3] = dc_ld128(sb + su1 + 16);
+        R.x[0][2] = dc_ld128(sb + su1);
+        R.x[0][3] = dc_ld128(sb + su1 + 16);
       }
       uint32_t a[16];
-      dc_frag_bf16<TT>(R, a);
-      dc_block_mma<TT>(d, a, R);
+      dc_frag_bf16(R.c, a);
+      dc_block_mma<TT>(d, a, R.x[0]);
     }
 #pragma unroll
     for (int c = 0; c < NACC; ++c) {
