@@ -275,27 +275,6 @@ bool make_tmap_t(CUtensorMap* m, const void* ptr, TmType t, uint64_t inner, uint
                  box_inner, box_outer, (int)swizzle128, (int)r);
   return r == CUDA_SUCCESS;
 }
-// 3-D tensor: dims[0] contiguous elements, dims[1] and dims[2] with byte strides strides[0], strides[1].
-bool make_tmap_3d(CUtensorMap* m, const void* ptr, TmType t, const uint64_t (&dims)[3], const uint64_t (&strides)[2],
-                  const uint32_t (&box)[3], bool swizzle128) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const CUtensorMapDataType dt = t == TmType::kBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                 : t == TmType::kU8  ? CU_TENSOR_MAP_DATA_TYPE_UINT8
-                                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-  cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
-  cuuint64_t st[2] = {strides[0], strides[1]};
-  cuuint32_t bx[3] = {box[0], box[1], box[2]};
-  cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = fn(m, dt, 3, const_cast<void*>(ptr), d, st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS && debug_on())
-    std::fprintf(stderr, "qlora: 3-D tensor map (ptr %p, dims %llu x %llu x %llu, box %u x %u x %u) -> %d\n", ptr,
-                 (unsigned long long)dims[0], (unsigned long long)dims[1], (unsigned long long)dims[2], box[0], box[1],
-                 box[2], (int)r);
-  return r == CUDA_SUCCESS;
-}
 bool make_tmap(CUtensorMap* m, const void* ptr, bool bf16, uint64_t inner, uint64_t outer,
                uint32_t box_inner, uint32_t box_outer, bool swizzle128 = true) {
   return make_tmap_t(m, ptr, bf16 ? TmType::kBf16 : TmType::kU8, inner, outer, inner, box_inner, box_outer,
