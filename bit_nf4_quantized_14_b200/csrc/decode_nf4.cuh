@@ -612,10 +612,11 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
     }
   };
 
-  // The flat stage sequence. At stage i: wait for this thread's copies of stage i, then a barrier of the
-  // consumer warps (every warp's copies of stage i landed; every warp is done with stage i - 1, whose slot
-  // the copies of stage i + R - 1 reuse), issue those copies, load the next stage's X words, compute.
-  DcCursor cc, ci, cx;
+  // The flat stage sequence. At stage i: load stage i's X words (their latency overlaps the waits), wait
+  // for this thread's copies of stage i, then a barrier of the consumer warps (every warp's copies of stage
+  // i landed; every warp is done with stage i - 1, whose slot the copies of stage i + R - 1 reuse), issue
+  // those copies, compute. One copy of the stage code: a smaller kernel keeps the instruction cache warm.
+  DcCursor cc, ci;
   cc.init(npa, pnb, pne);
   ci.init(npa, pnb, pne);
 #pragma unroll
@@ -623,24 +624,15 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
     issue(ci);
     ci.next(spp, npa, pnb, pne);
   }
-  cx = cc;
-  DcRegs<TT> ra, rb;
-  loadx(cx, ra);
-  cx.next(spp, npa, pnb, pne);
-  auto step = [&](DcRegs<TT>& cur, DcRegs<TT>& nxt) {
+  DcRegs<TT> rg;
+  while (cc.i < nmain) {
+    loadx(cc, rg);
     dc_cp_wait<kDcRing - 2>();
     dc_bar_consumers();
     issue(ci);
     ci.next(spp, npa, pnb, pne);
-    loadx(cx, nxt);
-    cx.next(spp, npa, pnb, pne);
-    stage(cc, cur);
+    stage(cc, rg);
     cc.next(spp, npa, pnb, pne);
-  };
-  while (cc.i < nmain) {
-    step(ra, rb);
-    if (cc.i >= nmain) break;
-    step(rb, ra);
   }
   dc_cp_wait<0>();
   if (p.u_only) {
