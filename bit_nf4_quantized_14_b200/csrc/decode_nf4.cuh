@@ -27,7 +27,7 @@
 //     permuted (the same permutation on both operands) so lane j's 16 elements are 16 j .. 16 j + 15;
 //   * the block constant c1_hat = fma(decode(e4m3), s2, mu) multiplies the fp32 result of each block's four
 //     MMAs; two helper warps (alternate stages) decode each stage's constants into a ring of shared-memory
-//     buffers ahead of the consumers, from raw bytes each loads three of its stages ahead;
+//     buffers ahead of the consumers;
 //   * at the end of each pass the 16 warps' partial sums meet in shared memory and are added in warp
 //     order (deterministic). A tiles come first: their sums, times s and rounded to bf16, are sU, which the
 //     CTA publishes with a per-call tag; a gather warp in every CTA waits for all of sU and copies it into
@@ -298,8 +298,7 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
     const int nnf = nmain - nfirst;
     if (nnf == 0) return;
     const float mu = __ldg(p.mu);
-    // Rows lane and lane + 32 of the pass; the raw E4M3 bytes and group scales of NF4 stage k sit in ring
-    // entry k % 3, loaded three stages before they are decoded.
+    // Rows lane and lane + 32 of the pass: the raw E4M3 bytes and group scales of NF4 stage k.
     struct Raw { uint32_t ew[2][4]; float sa[2], sz[2]; };
     auto fetch = [&](int k, Raw& f) {
       if (k >= nnf) return;
@@ -363,30 +362,24 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
         }
       }
     };
-    Raw ring[3];
-    fetch(sw, ring[0]);
-    fetch(sw + kDcScaleWarps, ring[1]);
-    fetch(sw + 2 * kDcScaleWarps, ring[2]);
+    // Fetch and decode in sequence (one copy of the code; the two warps between them stay ahead of the
+    // consumers by up to kDcCRing stages, which covers the load latency).
     bool go = true;
-    for (int k0 = sw; k0 < nnf && go; k0 += 3 * kDcScaleWarps) {
-#pragma unroll
-      for (int u = 0; u < 3; ++u) {
-        const int k = k0 + u * kDcScaleWarps;
-        if (k >= nnf) break;
-        // its buffer last held NF4 stage k - R: wait until every consumer warp has read it
-        if (k >= kDcCRing && lane == 0 &&
-            !mbar_wait(&cfree[k % kDcCRing], static_cast<uint32_t>(((k / kDcCRing) - 1) & 1)))
-          *abort_flag = 1;
-        __syncwarp();
-        if (*abort_flag) {
-          go = false;
-          break;
-        }
-        decode(k, ring[u]);
-        fetch(k + 3 * kDcScaleWarps, ring[u]);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&cready[k % kDcCRing]);
+    for (int k = sw; k < nnf && go; k += kDcScaleWarps) {
+      Raw r;
+      fetch(k, r);
+      // its buffer last held NF4 stage k - R: wait until every consumer warp has read it
+      if (k >= kDcCRing && lane == 0 &&
+          !mbar_wait(&cfree[k % kDcCRing], static_cast<uint32_t>(((k / kDcCRing) - 1) & 1)))
+        *abort_flag = 1;
+      __syncwarp();
+      if (*abort_flag) {
+        go = false;
+        break;
       }
+      decode(k, r);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&cready[k % kDcCRing]);
     }
     return;
   }
