@@ -41,6 +41,8 @@
 // unwinds without further waits. Named barriers among the consumer warps are reached on every path.
 #pragma once
 
+#include <type_traits>
+
 #include "codec.cuh"
 #include "common.cuh"
 
@@ -433,10 +435,10 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
   // NF4 rows 4 w .. 4 w + 3 of the pass (512 B each, piece pc of row rho at rho * 512 + (pc ^ (rho & 7)) * 16),
   // or A row w (2 KB, piece pc at w * 2048 + (pc ^ (w & 7)) * 16). Pieces outside the matrix are zero-filled
   // without a read.
-  auto issue = [&](const DcCursor& c) {
+  auto issue = [&](const DcCursor& c, auto nf4_only) {
     if (c.i < nmain) {
       const uint32_t slot = slot_addr(c.i % kDcRing);
-      if (c.ps.isA) {
+      if (!decltype(nf4_only)::value && c.ps.isA) {
 #pragma unroll
         for (int ra = 0; ra < kDcARowsPw; ++ra) {
           const int rho = kDcARowsPw * w + ra;
@@ -498,7 +500,7 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
   float acc[PT][NACC];
   bool live = true;
   int knf = 0;                                      // NF4 stages computed so far (the constants ring index)
-  auto stage = [&](const DcCursor& c, DcRegs<TT>& R) {
+  auto stage = [&](const DcCursor& c, DcRegs<TT>& R, auto is_a) {
     const DcPass& ps = c.ps;
     if (c.st == 0) {
 #pragma unroll
@@ -508,7 +510,7 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
     }
     const uint32_t slot = slot_addr(c.i % kDcRing);
     if (live && *abort_flag) live = false;
-    if (ps.isA) {
+    if constexpr (decltype(is_a)::value) {
 #pragma unroll
       for (int b = 0; b < kDcBpw; ++b) {
         const int bw = kDcBpw * w + b;              // block of the stage
@@ -591,7 +593,7 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
       float sum = 0.0f;
 #pragma unroll
       for (int ww = 0; ww < kDcWarps; ++ww) sum += *dc_red(lut, (ww * prow + ro) * T + t);
-      if (ps.isA) {                                 // sU = bf16(s * X A^T): column = A row
+      if constexpr (decltype(is_a)::value) {        // sU = bf16(s * X A^T): column = A row
         const int arow = (sh.a0 + ps.first) * 16 + ro;
         if (arow < p.r) p.U[static_cast<int64_t>(t) * p.r + arow] = __float2bfloat16_rn(p.s * sum);
       } else {
@@ -599,32 +601,45 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
       }
     }
     dc_bar_consumers();
-    if (ps.isA && threadIdx.x == 0) {               // this A tile's piece of sU is complete and visible
+    if (decltype(is_a)::value && threadIdx.x == 0) {   // this A tile's piece of sU is complete and visible
       __threadfence();
       st_release_u64(p.tags + sh.a0 + ps.first, p.seq);
     }
   };
 
-  // The flat stage sequence. At stage i: load stage i's X words (their latency overlaps the waits), wait
-  // for this thread's copies of stage i, then a barrier of the consumer warps (every warp's copies of stage
-  // i landed; every warp is done with stage i - 1, whose slot the copies of stage i + R - 1 reuse), issue
-  // those copies, compute. One copy of the stage code: a smaller kernel keeps the instruction cache warm.
+  // The flat stage sequence, A stages first, then NF4 stages (two loops, each with only its own code). At
+  // stage i: load stage i's X words (their latency overlaps the waits), wait for this thread's copies of
+  // stage i, then a barrier of the consumer warps (every warp's copies of stage i landed; every warp is done
+  // with stage i - 1, whose slot the copies of stage i + R - 1 reuse), issue those copies, compute.
+  using kA = std::integral_constant<bool, true>;      // stage(): an A stage
+  using kNF4 = std::integral_constant<bool, false>;   // stage(): an NF4 stage
+  using kAnyStage = std::integral_constant<bool, false>;   // issue(): A or NF4
+  using kNF4Only = std::integral_constant<bool, true>;     // issue(): NF4 only
   DcCursor cc, ci;
   cc.init(npa, pnb, pne);
   ci.init(npa, pnb, pne);
 #pragma unroll
   for (int i = 0; i < kDcRing - 1; ++i) {
-    issue(ci);
+    issue(ci, kAnyStage{});
     ci.next(spp, npa, pnb, pne);
   }
   DcRegs<TT> rg;
-  while (cc.i < nmain) {
+  while (cc.i < nfirst) {
     loadx(cc, rg);
     dc_cp_wait<kDcRing - 2>();
     dc_bar_consumers();
-    issue(ci);
+    issue(ci, kAnyStage{});
     ci.next(spp, npa, pnb, pne);
-    stage(cc, rg);
+    stage(cc, rg, kA{});
+    cc.next(spp, npa, pnb, pne);
+  }
+  while (cc.i < nmain) {                            // every stage issued from here on is an NF4 stage
+    loadx(cc, rg);
+    dc_cp_wait<kDcRing - 2>();
+    dc_bar_consumers();
+    issue(ci, kNF4Only{});
+    ci.next(spp, npa, pnb, pne);
+    stage(cc, rg, kNF4{});
     cc.next(spp, npa, pnb, pne);
   }
   dc_cp_wait<0>();
