@@ -13,20 +13,22 @@
 //     (the adapter projection), in tiles of 16 rows, are split into contiguous ranges, one per CTA (an A
 //     tile weighs 4 NF4 tiles: bf16 against 4-bit); each CTA contracts its tiles over the whole K, so no
 //     partial sum crosses CTAs;
-//   * passes of up to 4 tiles (2 for more than 8 tokens), each a sequence of stages of 16 blocks (1024
-//     contraction elements); consumer warp w takes block w of every stage. A stage (64 rows x 512 B of
-//     codes, or 16 A rows x 2 KB) comes into a ring of 4 shared-memory slots by cp.async three stages
-//     ahead, ~96 KB per SM in flight without holding registers: each warp copies 4 whole 512-byte row
-//     segments (contiguous runs, which HBM serves a quarter faster than 32-byte pieces of 64 rows), one
-//     named barrier per stage publishes the slot, and 16-byte pieces are XOR-swizzled by row so the
-//     fragment loads are free of bank conflicts;
+//   * passes of up to 4 tiles (2 above 8 tokens), each a sequence of stages of 16 blocks (1024 contraction
+//     elements); each of the 8 consumer warps takes 2 blocks of every stage (fewer, fuller warps: less
+//     per-stage bookkeeping per weight). A stage (64 rows x 512 B of codes, or 16 A rows x 2 KB) comes into a ring of 4
+//     shared-memory slots by cp.async three stages ahead, ~96 KB per SM in flight without holding
+//     registers: each warp copies 8 whole 512-byte row segments (contiguous runs, which HBM serves a quarter
+//     faster than 32-byte pieces of 64 rows), one named barrier per stage publishes the slot, and 16-byte
+//     pieces are XOR-swizzled by row so the fragment loads are free of bank conflicts. The A stages and the
+//     NF4 stages run in two loops, each holding only its own code: the stage code is large, and keeping one
+//     copy of it per loop keeps the instruction cache warm;
 //   * mma.sync m16n8k16 with the weight as the 16-row A operand and X as the 8-token B operand. The A
-//     fragments come from code bytes: prmt forms (byte << 8 | lane * 4) and one shared-memory load fetches
-//     the bf16 pair (level[hi], level[lo]) from a 256-entry table replicated per lane (entries 256 B
-//     apart: no further arithmetic, no bank conflicts). Inside each 64-element block the MMA's k index is
+//     fragments come from code bytes: one prmt forms the whole shared address (1 << 16 | byte << 8 |
+//     lane * 4) and one shared-memory load fetches the bf16 pair (level[hi], level[lo]) from a 256-entry
+//     table at shared address 64 KB, replicated per lane (entries 256 B apart: no bank conflicts). Inside each 64-element block the MMA's k index is
 //     permuted (the same permutation on both operands) so lane j's 16 elements are 16 j .. 16 j + 15;
 //   * the block constant c1_hat = fma(decode(e4m3), s2, mu) multiplies the fp32 result of each block's four
-//     MMAs; two helper warps (alternate stages) decode each stage's constants into a ring of shared-memory
+//     MMAs (run as two chains of two); two helper warps (alternate stages) decode each stage's constants into a ring of shared-memory
 //     buffers ahead of the consumers;
 //   * at the end of each pass the 16 warps' partial sums meet in shared memory and are added in warp
 //     order (deterministic). A tiles come first: their sums, times s and rounded to bf16, are sU, which the
@@ -253,9 +255,28 @@ __device__ __forceinline__ void dc_block_mma(float (&d)[TT == 16 ? 8 : 4], const
   }
 }
 
+// The same contraction as dc_block_mma with the four MMA steps in two chains (steps 0, 2 into d0 and 1, 3
+// into d1), so two MMA latencies are in flight instead of one; the caller adds d0 + d1.
+template <int TT>
+__device__ __forceinline__ void dc_block_mma2(float (&d0)[TT == 16 ? 8 : 4], float (&d1)[TT == 16 ? 8 : 4],
+                                              const uint32_t (&a)[16], const uint4 (&x)[TT / 4]) {
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    float (&d)[TT == 16 ? 8 : 4] = (s & 1) ? d1 : d0;
+    const uint4& xv = x[s >> 1];
+    dc_mma(d[0], d[1], d[2], d[3], a[4 * s], a[4 * s + 1], a[4 * s + 2], a[4 * s + 3], dc_word(xv, 2 * (s & 1)),
+           dc_word(xv, 2 * (s & 1) + 1));
+    if constexpr (TT == 16) {
+      const uint4& xw = x[2 + (s >> 1)];
+      dc_mma(d[4], d[5], d[6], d[7], a[4 * s], a[4 * s + 1], a[4 * s + 2], a[4 * s + 3], dc_word(xw, 2 * (s & 1)),
+             dc_word(xw, 2 * (s & 1) + 1));
+    }
+  }
+}
+
 template <int TT>
 __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecParams p, const CodebookArg cb) {
-  constexpr int PT = TT == 16 ? 2 : kDcMaxTiles;      // tiles per pass
+  constexpr int PT = TT == 16 ? 2 : kDcMaxTiles;      // tiles per pass (4 spill at 16 tokens: slower)
   constexpr int NACC = TT == 16 ? 8 : 4;
   extern __shared__ __align__(1024) uint8_t dc_smem[];
   uint8_t* dsm = dc_smem;
@@ -563,13 +584,13 @@ __global__ void __launch_bounds__(kDcThreads, 1) nf4_decode_kernel(const DecPara
             a[10] = dc_pair<1>(c0.y, lanebyte); a[11] = dc_pair<1>(c1.y, lanebyte);
             a[12] = dc_pair<2>(c0.y, lanebyte); a[13] = dc_pair<2>(c1.y, lanebyte);
             a[14] = dc_pair<3>(c0.y, lanebyte); a[15] = dc_pair<3>(c1.y, lanebyte);
-            float d[NACC];
+            float d0[NACC], d1[NACC];
 #pragma unroll
-            for (int e = 0; e < NACC; ++e) d[e] = 0.0f;
-            dc_block_mma<TT>(d, a, R.x[b]);
+            for (int e = 0; e < NACC; ++e) d0[e] = d1[e] = 0.0f;
+            dc_block_mma2<TT>(d0, d1, a, R.x[b]);
 #pragma unroll
             for (int e = 0; e < NACC; ++e)
-              acc[q][e] = __fmaf_rn((e & 2) ? cs[b][q].y : cs[b][q].x, d[e], acc[q][e]);
+              acc[q][e] = __fmaf_rn((e & 2) ? cs[b][q].y : cs[b][q].x, d0[e] + d1[e], acc[q][e]);
           }
         }
       }
