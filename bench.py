@@ -627,7 +627,7 @@ def secondary_figures(q, device, reps=20, warmup=3):
 DECODE_TOKENS = (1, 4, 16)
 DECODE_WORKLOAD = ("LLaMA-65B-shaped frozen NF4 linears (N x K = 8192x8192, 22016x8192, 8192x22016), "
                    "forward only at T = 1, 4, 16 tokens, r = 64, alpha = 16")
-SWEEP_SIZES = tuple(2 ** e for e in (20, 22, 24, 26, 28, 30))
+SWEEP_SIZES = tuple(2 ** e for e in (20, 22, 24, 26, 28, 30, 31))
 
 
 def gemv_bytes(T, N, K, r):
@@ -790,17 +790,20 @@ def run_decode(args):
 
 def run_codec_sweep(args):
     import torch
-    import synth
     import bit_nf4_quantized_14_b200 as q
     peaks, kind = load_peaks()
     device = torch.device("cuda", 0)
     flush = L2Flush(device)
-    chunk = 1 << 28          # the largest sizes are concatenations of independent 2^28-element sweep tensors
+    # the sweep tensor is drawn on the device (seeded torch generator; rows of 4096, sigma_row ~ U(0.005,
+    # 0.05), 0.1 % x10 outliers), in independent 2^28-element pieces: 2^31 elements in seconds, not minutes
+    chunk = 1 << 28
     nmax = max(SWEEP_SIZES)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(50)
     x = torch.empty(nmax, dtype=torch.float32, device=device)
     for c in range(0, nmax, chunk):
         m = min(chunk, nmax - c)
-        x[c:c + m] = torch.from_numpy(synth.sweep_f32(m, seed=50, tensor_id=c // chunk)).to(device)
+        x[c:c + m] = device_sweep(m, gen)
     xb = x.to(torch.bfloat16)
     cases = []
     for n in SWEEP_SIZES:
@@ -835,7 +838,8 @@ def run_codec_sweep(args):
                       "warmup": args.warmup, "higher_is_better": True, "dtype": "f32/bf16 in, u8 + e4m3 out",
                       "data": "synthetic",
                       "config": {"workload": "sweep tensors: rows of 4096, sigma_row ~ U(0.005, 0.05), 0.1 % x10 "
-                                             "outliers; sizes 2^20..2^30 (2^30 = four 2^28 sweeps)",
+                                             "outliers, drawn on the device; sizes 2^20..2^31 (2^30 and 2^31 = independent 2^28 "
+                                             "pieces)",
                                  "l2": L2_NOTE},
                       "roofline": {"bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"],
                                    "peak_source": f"{kind} (HBM copy)"},
